@@ -1,0 +1,170 @@
+"""CPU oracle for the FP8 W8A8 linear layer -- TEST INFRASTRUCTURE ONLY.
+
+Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline / reference leg
+of ``bench.py`` may import this package.  The product library never does, and
+the oracle shares no code with it: the arithmetic lives in ``fp8_oracle.c``
+(plain C, scalar loops, fp64 GEMM) and this module only marshals numpy arrays.
+
+Every function cites the passage it follows in ``fp8_oracle.c``.  Parity is
+pinned by ``tests/test_oracle_*.py`` against values the pages fix (E4M3 max 448,
+E5M2 max 57344), closed forms, library casts and hand-computed cases.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+E4M3, E5M2 = 0, 1
+SCALE_FP32, SCALE_UE8M0 = 0, 1
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        u8p = ctypes.POINTER(ctypes.c_uint8)
+        L.orc_decode.restype = ctypes.c_double
+        L.orc_decode.argtypes = [ctypes.c_uint8, ctypes.c_int]
+        L.orc_encode.restype = ctypes.c_uint8
+        L.orc_encode.argtypes = [ctypes.c_float, ctypes.c_int]
+        L.orc_fmax.restype = ctypes.c_double
+        L.orc_fmax.argtypes = [ctypes.c_int]
+        L.orc_scale_from_amax.restype = ctypes.c_float
+        L.orc_scale_from_amax.argtypes = [ctypes.c_float, ctypes.c_int, ctypes.c_int]
+        L.orc_round_bf16.restype = ctypes.c_uint16
+        L.orc_round_bf16.argtypes = [ctypes.c_double]
+        vp = ctypes.c_void_p
+        i64 = ctypes.c_int64
+        L.orc_act_quant.restype = None
+        L.orc_act_quant.argtypes = [vp, i64, i64, i64, i64, ctypes.c_int, ctypes.c_int, vp, vp]
+        L.orc_weight_quant_block.restype = None
+        L.orc_weight_quant_block.argtypes = [vp, i64, i64, i64, ctypes.c_int, ctypes.c_int, vp, vp]
+        L.orc_tensor_quant.restype = None
+        L.orc_tensor_quant.argtypes = [vp, i64, ctypes.c_int, ctypes.c_int, vp, vp]
+        L.orc_gemm_rows.restype = None
+        L.orc_gemm_rows.argtypes = [vp, vp, vp, vp, i64, i64, vp, i64, vp, vp]
+        L.orc_grouped_gemm_rows.restype = None
+        L.orc_grouped_gemm_rows.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp, i64, vp, vp]
+        del u8p
+        _lib = L
+    return _lib
+
+
+def _ptr(a: np.ndarray) -> int:
+    assert a.flags["C_CONTIGUOUS"], "oracle arrays must be C-contiguous"
+    return a.ctypes.data
+
+
+def _bf16_bits(x) -> np.ndarray:
+    """Accept a uint16 array of bf16 bit patterns or a torch bf16 CPU tensor."""
+    if isinstance(x, np.ndarray):
+        assert x.dtype == np.uint16
+        return np.ascontiguousarray(x)
+    import torch
+    assert x.dtype == torch.bfloat16 and x.device.type == "cpu"
+    return np.ascontiguousarray(x.contiguous().view(torch.int16).numpy().view(np.uint16))
+
+
+# ----------------------------------------------------------------- codec
+def decode(code: int, fmt: int = E4M3) -> float:
+    return lib().orc_decode(code & 0xFF, fmt)
+
+
+def encode(x: float, fmt: int = E4M3) -> int:
+    return int(lib().orc_encode(x, fmt))
+
+
+def fmax(fmt: int = E4M3) -> float:
+    return lib().orc_fmax(fmt)
+
+
+def scale_from_amax(amax: float, fmt: int = E4M3, scale_fmt: int = SCALE_FP32) -> float:
+    return float(lib().orc_scale_from_amax(amax, fmt, scale_fmt))
+
+
+def decode_table(fmt: int = E4M3) -> np.ndarray:
+    """fp64 value of each of the 256 codes (NaN where the code is NaN)."""
+    return np.array([decode(c, fmt) for c in range(256)], dtype=np.float64)
+
+
+def round_bf16(v: np.ndarray) -> np.ndarray:
+    """fp64 -> bf16 bit patterns, one direct round-to-nearest-even."""
+    f = lib().orc_round_bf16
+    flat = np.asarray(v, dtype=np.float64).ravel()
+    out = np.fromiter((f(float(t)) for t in flat), dtype=np.uint16, count=flat.size)
+    return out.reshape(np.shape(v))
+
+
+# ------------------------------------------------------------ quantisers
+def act_quant(x, group: int = 128, fmt: int = E4M3, scale_fmt: int = SCALE_FP32):
+    """x: [M, K] bf16 (bits or torch tensor) -> (q uint8 [M, K], s fp32 [M, ceil(K/group)])."""
+    xb = _bf16_bits(x)
+    M, K = xb.shape
+    ng = (K + group - 1) // group
+    q = np.empty((M, K), dtype=np.uint8)
+    s = np.empty((M, ng), dtype=np.float32)
+    lib().orc_act_quant(_ptr(xb), M, K, K, group, fmt, scale_fmt, _ptr(q), _ptr(s))
+    return q, s
+
+
+def weight_quant(w, block: int = 128, fmt: int = E4M3, scale_fmt: int = SCALE_FP32):
+    """w: [N, K] bf16 -> (q uint8 [N, K], s_inv fp32 [ceil(N/b), ceil(K/b)]); block=0 is per-tensor."""
+    wb = _bf16_bits(w)
+    N, K = wb.shape
+    q = np.empty((N, K), dtype=np.uint8)
+    if block == 0:
+        s = np.empty((1,), dtype=np.float32)
+        lib().orc_tensor_quant(_ptr(wb), N * K, fmt, scale_fmt, _ptr(q), _ptr(s))
+        return q, s
+    s = np.empty(((N + block - 1) // block, (K + block - 1) // block), dtype=np.float32)
+    lib().orc_weight_quant_block(_ptr(wb), N, K, block, fmt, scale_fmt, _ptr(q), _ptr(s))
+    return q, s
+
+
+def tensor_quant(x, fmt: int = E4M3, scale_fmt: int = SCALE_FP32):
+    """Per-tensor quantisation of any bf16 array -> (q uint8 same shape, s fp32 [1])."""
+    xb = _bf16_bits(x)
+    q = np.empty(xb.shape, dtype=np.uint8)
+    s = np.empty((1,), dtype=np.float32)
+    lib().orc_tensor_quant(_ptr(xb), xb.size, fmt, scale_fmt, _ptr(q), _ptr(s))
+    return q, s
+
+
+# ------------------------------------------------------------------ GEMM
+def gemm_rows(qa, sa, qw, sw, rows=None):
+    """fp64 block-scaled GEMM on the given rows -> (y [nr, N] fp64, bound [nr, N] fp64)."""
+    qa = np.ascontiguousarray(qa, dtype=np.uint8)
+    qw = np.ascontiguousarray(qw, dtype=np.uint8)
+    sa = np.ascontiguousarray(sa, dtype=np.float32)
+    sw = np.ascontiguousarray(sw, dtype=np.float32)
+    M, K = qa.shape
+    N = qw.shape[0]
+    assert K % 128 == 0 and qw.shape[1] == K
+    rows = np.arange(M, dtype=np.int64) if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    y = np.empty((rows.size, N), dtype=np.float64)
+    b = np.empty((rows.size, N), dtype=np.float64)
+    lib().orc_gemm_rows(_ptr(qa), _ptr(sa), _ptr(qw), _ptr(sw), N, K, _ptr(rows), rows.size, _ptr(y), _ptr(b))
+    return y, b
+
+
+def grouped_gemm_rows(qa, sa, qw, sw, offsets, rows):
+    """Grouped GEMM on selected rows.  qw: [E, N, K], sw: [E, ceil(N/128), K/128], offsets int32 [E+1]."""
+    qa = np.ascontiguousarray(qa, dtype=np.uint8)
+    qw = np.ascontiguousarray(qw, dtype=np.uint8)
+    sa = np.ascontiguousarray(sa, dtype=np.float32)
+    sw = np.ascontiguousarray(sw, dtype=np.float32)
+    off = np.ascontiguousarray(offsets, dtype=np.int32)
+    E, N, K = qw.shape
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    y = np.empty((rows.size, N), dtype=np.float64)
+    b = np.empty((rows.size, N), dtype=np.float64)
+    lib().orc_grouped_gemm_rows(_ptr(qa), _ptr(sa), _ptr(qw), _ptr(sw), _ptr(off), E, N, K,
+                                _ptr(rows), rows.size, _ptr(y), _ptr(b))
+    return y, b

@@ -1,0 +1,292 @@
+/*
+ * fp8_oracle.c -- plain, slow, scalar CPU oracle for the FP8 W8A8 linear layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product library links, loads or
+ * calls this file; only the tests, the smoke check and the CPU baseline leg of
+ * the benchmark do.  It shares no code, header, table or constant generator with
+ * the CUDA library: every formula below is written out again from the pages.
+ *
+ * Sources (page title, then the section the step follows):
+ *  [P1] "ROCm 7 原生 FP8/MXFP8 ... AITER" (devpress.csdn.net), section 1.1 table
+ *       (E4M3 range +-448, E5M2 range +-57344) and section 4.3 "延迟缩放"
+ *       (divide by the scale, clamp to +-448, cast to float8_e4m3fn).
+ *  [P2] "LLM 推理的 FP8 混合精度工程 2026" (blog.lonae.com), section 2, the
+ *       quantisation operator Q(x) = clamp(round(x*s), -Fmax, Fmax) * s^-1 with
+ *       Fmax = 448 (E4M3) / 57344 (E5M2); section 3, FP32 accumulation of FP8
+ *       products.
+ *  [P3] "FP8 推理" (luoboask.github.io), "Dynamic Scaling": FP8 = FP32 / scale,
+ *       scale = max(|tensor|) / 448.
+ *  [P4] "FP8 推理提速 83.6%: DeepSeek-V3 在 AMD MI250 上的完整落地指南" (xdnf.cn),
+ *       "FP8 权重转换命令与关键配置参数" (e4m3 weights with 128x128 block
+ *       scale_inv; scale_fmt ue8m0) and "运行时" (act_quant per token per 128
+ *       channels, then fp8_gemm(x, scale, weight, weight.scale)).
+ *  [P5] "量化：FP8 与混合精度推理" (charles2530.github.io), "FP8 也需要 scale":
+ *       x_fp8 = FP8Cast(x / s), x_hat = s * x_fp8.
+ *
+ * Readings taken where the pages are silent (each one is listed in the design doc):
+ *  - the scale divides (x / s), it is stored as the dequantisation multiplier;
+ *  - the division x / s is one IEEE fp32 division, then round-to-nearest-even
+ *    to FP8 with saturation to +-Fmax (no Inf is ever produced);
+ *  - s = max(fl32(amax / Fmax), 2^-126); ue8m0 rounds fl32(amax / Fmax) up to
+ *    a power of two 2^e with e >= -126;
+ *  - a negative value that rounds to zero keeps its sign (code 0x80);
+ *  - NaN inputs are ignored by amax and encode as 0x7F.
+ *
+ * Build: gcc -O1 -std=c99 -fPIC -shared -ffp-contract=off (no fast-math), so
+ * every float operation below is one correctly rounded IEEE operation.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stddef.h>
+
+#define ORC_E4M3 0
+#define ORC_E5M2 1
+#define ORC_SCALE_FP32 0
+#define ORC_SCALE_UE8M0 1
+
+/* ------------------------------------------------------------------ codec */
+
+/* Decode one FP8 code.  [P1] 1.1 / [P2] 2: E4M3 = 1 sign, 4 exponent (bias 7),
+ * 3 mantissa bits, largest finite 448, no infinity, S.1111.111 is NaN.
+ * E5M2 = 1 sign, 5 exponent (bias 15), 2 mantissa bits, largest finite 57344,
+ * exponent 31 is Inf (mantissa 0) or NaN. */
+double orc_decode(uint8_t code, int fmt)
+{
+    int neg = code >> 7;
+    double v;
+    if (fmt == ORC_E4M3) {
+        int e = (code >> 3) & 15, m = code & 7;
+        if (e == 15 && m == 7) return NAN;
+        if (e == 0) v = ldexp((double)m, -9);            /* (m/8) * 2^(1-7)   */
+        else        v = ldexp((double)(8 + m), e - 10);  /* (1+m/8) * 2^(e-7) */
+    } else {
+        int e = (code >> 2) & 31, m = code & 3;
+        if (e == 31) return m == 0 ? (neg ? -INFINITY : INFINITY) : NAN;
+        if (e == 0) v = ldexp((double)m, -16);           /* (m/4) * 2^(1-15)  */
+        else        v = ldexp((double)(4 + m), e - 17);  /* (1+m/4) * 2^(e-15) */
+    }
+    return neg ? -v : v;
+}
+
+/* Largest finite code below the sign bit: 0x7E (448) for E4M3, 0x7B (57344)
+ * for E5M2.  Non-negative finite codes are 0 .. top and increase with the code. */
+static int top_code(int fmt) { return fmt == ORC_E4M3 ? 0x7E : 0x7B; }
+
+double orc_fmax(int fmt) { return orc_decode((uint8_t)top_code(fmt), fmt); }
+
+/* Values of the non-negative finite codes 0 .. top of each format, filled once
+ * by the decoder above (no constants are typed in). */
+static double g_tab[2][128];
+static int g_tab_ready[2];
+
+static const double *value_table(int fmt)
+{
+    if (!g_tab_ready[fmt]) {
+        for (int c = 0; c <= top_code(fmt); ++c) g_tab[fmt][c] = orc_decode((uint8_t)c, fmt);
+        g_tab_ready[fmt] = 1;
+    }
+    return g_tab[fmt];
+}
+
+/* Encode one fp32 value: the nearest FP8 value, ties to the code with an even
+ * mantissa, anything at or beyond Fmax (including Inf) clamps to Fmax ([P1] 4.3
+ * clamp-then-cast, [P2] 2 clamp(round(.))).  A binary search finds the two
+ * neighbouring table values; the distances are exact in double. */
+uint8_t orc_encode(float x, int fmt)
+{
+    if (isnan(x)) return 0x7F;
+    uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    double a = fabs((double)x);
+    int top = top_code(fmt);
+    const double *tab = value_table(fmt);
+    if (a >= tab[top]) return (uint8_t)(sign | top);
+    int lo = 0, hi = top;                  /* invariant: tab[lo] <= a < tab[hi] */
+    while (hi - lo > 1) {
+        int mid = (lo + hi) / 2;
+        if (tab[mid] <= a) lo = mid; else hi = mid;
+    }
+    double dlo = a - tab[lo];              /* exact: Sterbenz, or tab[lo] == 0 */
+    double dhi = tab[hi] - a;
+    int c;
+    if (dlo < dhi) c = lo;
+    else if (dhi < dlo) c = hi;
+    else c = (lo & 1) ? hi : lo;           /* tie: even mantissa LSB */
+    return (uint8_t)(sign | c);
+}
+
+/* ------------------------------------------------------------------ scales */
+
+/* Group / block / tensor scale from its amax.  [P3] Dynamic Scaling:
+ * scale = amax / Fmax.  FP32 format: the quotient in IEEE fp32, floored at
+ * 2^-126 so an all-zero group never divides by zero.  UE8M0 ([P4] scale_fmt):
+ * the same quotient rounded UP to a power of two, exponent >= -126. */
+float orc_scale_from_amax(float amax, int fmt, int scale_fmt)
+{
+    float fmax = (float)orc_fmax(fmt);
+    float v = amax / fmax;
+    if (scale_fmt == ORC_SCALE_FP32) {
+        return v < 0x1p-126f ? 0x1p-126f : v;
+    }
+    int e;
+    if (v == 0.0f) {
+        e = -126;
+    } else {
+        int p;
+        double m = frexp((double)v, &p);   /* v = m * 2^p, m in [0.5, 1) */
+        e = (m == 0.5) ? p - 1 : p;        /* ceil(log2 v) */
+        if (e < -126) e = -126;
+    }
+    return ldexpf(1.0f, e);
+}
+
+/* bf16 bit pattern -> fp32 (exact: bf16 is the top half of an fp32). */
+static float bf16_to_f32(uint16_t h)
+{
+    union { uint32_t u; float f; } c;
+    c.u = (uint32_t)h << 16;
+    return c.f;
+}
+
+/* |x| max over a set of bf16 values; NaN never wins a comparison. */
+static float amax_accum(float amax, float x)
+{
+    float a = fabsf(x);
+    return a > amax ? a : amax;
+}
+
+/* --------------------------------------------------------------- quantisers */
+
+/* Per-token, per-group activation quantisation ([P4] 运行时 act_quant; [P2] 4
+ * per-block activation scales of 128 elements).  x is [M][ldx] bf16, q is
+ * [M][K] codes, s is [M][ceil(K/group)] scales.  The last group of a row may
+ * be short; its amax covers only the valid elements. */
+void orc_act_quant(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
+                   int64_t group, int fmt, int scale_fmt,
+                   uint8_t *q, float *s)
+{
+    int64_t ng = (K + group - 1) / group;
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t g = 0; g < ng; ++g) {
+            int64_t k0 = g * group, k1 = k0 + group < K ? k0 + group : K;
+            float amax = 0.0f;
+            for (int64_t k = k0; k < k1; ++k)
+                amax = amax_accum(amax, bf16_to_f32(x[m * ldx + k]));
+            float sc = orc_scale_from_amax(amax, fmt, scale_fmt);
+            s[m * ng + g] = sc;
+            for (int64_t k = k0; k < k1; ++k) {
+                float t = bf16_to_f32(x[m * ldx + k]) / sc;   /* one IEEE division */
+                q[m * K + k] = orc_encode(t, fmt);
+            }
+        }
+    }
+}
+
+/* 128x128 block weight quantisation ([P4] FP8 权重转换: e4m3 weights with a
+ * 128x128 block scale_inv).  w is [N][K] bf16 (row stride K), q is [N][K],
+ * s_inv is [ceil(N/block)][ceil(K/block)]. */
+void orc_weight_quant_block(const uint16_t *w, int64_t N, int64_t K, int64_t block,
+                            int fmt, int scale_fmt, uint8_t *q, float *s_inv)
+{
+    int64_t nbn = (N + block - 1) / block, nbk = (K + block - 1) / block;
+    for (int64_t bn = 0; bn < nbn; ++bn) {
+        for (int64_t bk = 0; bk < nbk; ++bk) {
+            int64_t n0 = bn * block, n1 = n0 + block < N ? n0 + block : N;
+            int64_t k0 = bk * block, k1 = k0 + block < K ? k0 + block : K;
+            float amax = 0.0f;
+            for (int64_t n = n0; n < n1; ++n)
+                for (int64_t k = k0; k < k1; ++k)
+                    amax = amax_accum(amax, bf16_to_f32(w[n * K + k]));
+            float sc = orc_scale_from_amax(amax, fmt, scale_fmt);
+            s_inv[bn * nbk + bk] = sc;
+            for (int64_t n = n0; n < n1; ++n)
+                for (int64_t k = k0; k < k1; ++k)
+                    q[n * K + k] = orc_encode(bf16_to_f32(w[n * K + k]) / sc, fmt);
+        }
+    }
+}
+
+/* Per-tensor quantisation ([P1] 1.2 OCP-FP8 one scale per tensor; [P3] scale =
+ * max(|tensor|)/448; [P2] Fmax 57344 for E5M2).  One scale for all n elements. */
+void orc_tensor_quant(const uint16_t *x, int64_t n, int fmt, int scale_fmt,
+                      uint8_t *q, float *s)
+{
+    float amax = 0.0f;
+    for (int64_t i = 0; i < n; ++i) amax = amax_accum(amax, bf16_to_f32(x[i]));
+    float sc = orc_scale_from_amax(amax, fmt, scale_fmt);
+    s[0] = sc;
+    for (int64_t i = 0; i < n; ++i) q[i] = orc_encode(bf16_to_f32(x[i]) / sc, fmt);
+}
+
+/* -------------------------------------------------------------------- GEMM */
+
+/* Block-scaled GEMM, selected rows ([P4] 运行时 fp8_gemm(x, scale, weight,
+ * weight.scale); [P5] x_hat = s * x_fp8; [P2] 3 FP32 accumulation):
+ *   y[m][n] = sum_k (dec(qa[m][k]) * sa[m][k/128]) * (dec(qw[n][k]) * sw[n/128][k/128])
+ * summed in fp64 in k order.  bound[m][n] = sum_k |a_k * w_k| (the tolerance
+ * scale).  rows lists the nr rows to compute; outputs are [nr][N]. */
+void orc_gemm_rows(const uint8_t *qa, const float *sa, const uint8_t *qw, const float *sw,
+                   int64_t N, int64_t K, const int64_t *rows, int64_t nr,
+                   double *y, double *bound)
+{
+    const int64_t nkb = K / 128;
+    for (int64_t i = 0; i < nr; ++i) {
+        int64_t m = rows[i];
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0, b = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                double a = orc_decode(qa[m * K + k], ORC_E4M3) * (double)sa[m * nkb + k / 128];
+                double w = orc_decode(qw[n * K + k], ORC_E4M3) *
+                           (double)sw[(n / 128) * nkb + k / 128];
+                acc += a * w;
+                b += fabs(a * w);
+            }
+            y[i * N + n] = acc;
+            bound[i * N + n] = b;
+        }
+    }
+}
+
+/* Grouped (MoE expert) GEMM, selected rows: row m belongs to the expert e with
+ * off[e] <= m < off[e+1] and uses that expert's weights qw[e] ([N][K]) and
+ * scales sw[e] ([N/128][K/128]).  Rows outside every group get y = 0. */
+void orc_grouped_gemm_rows(const uint8_t *qa, const float *sa, const uint8_t *qw,
+                           const float *sw, const int32_t *off, int64_t E,
+                           int64_t N, int64_t K, const int64_t *rows, int64_t nr,
+                           double *y, double *bound)
+{
+    const int64_t nkb = K / 128, nbn = (N + 127) / 128;
+    for (int64_t i = 0; i < nr; ++i) {
+        int64_t m = rows[i], e = -1;
+        for (int64_t j = 0; j < E; ++j)
+            if (off[j] <= m && m < off[j + 1]) { e = j; break; }
+        if (e < 0) {
+            for (int64_t n = 0; n < N; ++n) { y[i * N + n] = 0.0; bound[i * N + n] = 0.0; }
+            continue;
+        }
+        orc_gemm_rows(qa, sa, qw + e * N * K, sw + e * nbn * nkb, N, K, &m, 1,
+                      y + i * N, bound + i * N);
+    }
+}
+
+/* ---------------------------------------------------------------- rounding */
+
+/* Round a double straight to bf16 (8-bit significand), ties to even, with
+ * gradual underflow; no intermediate fp32 rounding.  Used to state the bf16
+ * output the oracle expects. */
+uint16_t orc_round_bf16(double v)
+{
+    union { uint32_t u; float f; } c;
+    if (isnan(v)) return 0x7FC0;
+    double a = fabs(v);
+    uint16_t sign = signbit(v) ? 0x8000 : 0;
+    if (a == 0.0) return sign;
+    int p;
+    frexp(a, &p);                          /* a in [2^(p-1), 2^p) */
+    int q = p - 1 - 7;                     /* quantum exponent for a normal bf16 */
+    if (q < -133) q = -133;                /* subnormal quantum 2^-133 */
+    double r = nearbyint(ldexp(a, -q));    /* exact scaling; RNE (default mode) */
+    double out = ldexp(r, q);
+    if (out > 0x1.FEp127) return sign | 0x7F80;   /* overflow -> Inf */
+    c.f = (float)out;                      /* exact: out is a bf16 value */
+    return (uint16_t)(sign | (c.u >> 16));
+}
