@@ -1,0 +1,437 @@
+"""Benchmark of the FP8 W8A8 linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill|decode|moe|sweep]
+                    [--impl ours|reference] [--no-rows]
+
+Default workload (the headline): the prefill-shaped linear, x bf16 4096 x 8192
+(1% outlier channels x20), W 28672 x 8192 as E4M3 with 128x128 fp32 block scales
+(quantised once, as the pages ship FP8 checkpoints).  One step = act_quant(x)
+(per token, per 128 channels, fp32 scales) + block-scaled FP8 GEMM, bf16 out.
+Metric: GEMM TFLOPS over the step (2*M*N*K per step); act_quant GB/s is reported
+beside it.  Inputs are larger than L2 (W alone is 235 MB), so no flush is needed.
+
+Under torchrun every rank runs its own token batch through the same layer (data
+parallel, no collective on the data path: weak scaling); the barrier and the
+max-over-ranks timing use torch.distributed.
+
+--impl reference times the CPU oracle (plain C, fp64 GEMM) on a bounded sample
+of the same workload on the host cores; only rank 0 runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "block-scaled FP8 GEMM TFLOPS (% dense FP8 peak); act_quant GB/s (% HBM peak)"
+FP8_OVER_BF16 = 2.0          # nominal dense FP8 / BF16 tensor throughput ratio on B200 (4.5 / 2.25 PF)
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
+
+
+# --------------------------------------------------------------------- helpers
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK), "fallback"
+
+
+def source_sha() -> str:
+    h = hashlib.sha256()
+    for f in ("gemm.cuh", "ptx.cuh", "quant.cuh", "fp8lin.cu"):
+        h.update(open(os.path.join(ROOT, "fp8_block_scaled_12_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel_key: str):
+    """Per-launch DRAM bytes of `kernel_key` from the committed ncu summary, if the
+    summary was taken on the current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.md")
+    if not os.path.exists(p):
+        return None
+    sha = source_sha()
+    for line in open(p):
+        m = re.match(r"\|\s*" + re.escape(kernel_key) + r"\s*\|\s*([0-9.eE+]+)\s*\|\s*([0-9a-f]+)\s*\|", line)
+        if m and m.group(2) == sha:
+            return float(m.group(1))
+    return None
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML in a background thread."""
+    REASONS = {
+        0x0000000000000004: "sw_power_cap", 0x0000000000000008: "hw_slowdown",
+        0x0000000000000020: "sw_thermal_slowdown", 0x0000000000000040: "hw_thermal_slowdown",
+        0x0000000000000080: "hw_power_brake_slowdown", 0x0000000000000002: "applications_clocks_setting",
+    }
+
+    def __init__(self, index: int, period_s: float = 0.01):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period, self._stop = period_s, threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# ------------------------------------------------------------------ workloads
+def setup_prefill(dev, rank):
+    import torch
+    import fp8_block_scaled_12_b200 as F
+    import synth
+    p = synth.PREFILL.params
+    M, N, K = p["M"], p["N"], p["K"]
+    ch = synth.outlier_channels(K, synth.n_outliers(K, p["outlier_frac"]), seed=0)
+    x = synth.activations(M, K, seed=rank, outliers=ch, factor=p["factor"], device=dev)
+    w = synth.weights(N, K, p["w_std"], seed=0, device=dev)
+    qw, sw = F.weight_quant(w)
+    del w
+    qa = torch.empty((M, K), dtype=torch.uint8, device=dev)
+    sa = torch.empty((M, K // 128), dtype=torch.float32, device=dev)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    torch.cuda.synchronize()
+    return dict(M=M, N=N, K=K, x=x, qa=qa, sa=sa, qw=qw, sw=sw, y=y, F=F, desc=synth.PREFILL.desc)
+
+
+def run_ours(args, world, rank, local):
+    import torch
+    import torch.distributed as dist
+    dev = torch.device(f"cuda:{local}")
+    torch.cuda.set_device(dev)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    peaks, peak_src = load_peaks()
+    if args.workload != "prefill":
+        return run_other(args, world, rank, dev, peaks, peak_src)
+
+    S = setup_prefill(dev, rank)
+    F, M, N, K = S["F"], S["M"], S["N"], S["K"]
+    stream = torch.cuda.current_stream()
+    flops = 2.0 * M * N * K
+
+    def step():
+        F.fp8_act_quant(S["x"], S["qa"], S["sa"], stream=stream)
+        F.fp8_block_gemm(S["qa"], S["sa"], S["qw"], S["sw"], S["y"], stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert F.fp8_device_error() == 0
+
+    # -------- timed region: inputs resident in HBM
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t0.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            F.fp8_act_quant(S["x"], S["qa"], S["sa"], stream=stream)
+            ev[i][1].record(stream)
+            F.fp8_block_gemm(S["qa"], S["sa"], S["qw"], S["sw"], S["y"], stream=stream)
+            ev[i][2].record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = t0.elapsed_time(t1)
+    aq_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    gm_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    assert F.fp8_device_error() == 0
+
+    # -------- end to end through the public API with host buffers
+    x_host = S["x"].cpu().pin_memory()
+    y_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    xd = torch.empty_like(S["x"])
+    for _ in range(max(1, args.warmup // 2)):
+        xd.copy_(x_host, non_blocking=True)
+        F.fp8_act_quant(xd, S["qa"], S["sa"], stream=stream)
+        F.fp8_block_gemm(S["qa"], S["sa"], S["qw"], S["sw"], S["y"], stream=stream)
+        y_host.copy_(S["y"], non_blocking=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.steps):
+        xd.copy_(x_host, non_blocking=True)
+        F.fp8_act_quant(xd, S["qa"], S["sa"], stream=stream)
+        F.fp8_block_gemm(S["qa"], S["sa"], S["qw"], S["sw"], S["y"], stream=stream)
+        y_host.copy_(S["y"], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+
+    if world > 1:
+        t = torch.tensor([ms, e2e_ms, aq_ms, gm_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, e2e_ms, aq_ms, gm_ms = t.tolist()
+
+    tflops = flops * world * args.steps / (ms * 1e-3) / 1e12
+    e2e_tflops = flops * world * args.steps / (e2e_ms * 1e-3) / 1e12
+    gemm_tflops = flops / (gm_ms * 1e-3) / 1e12
+    aq_bytes = M * K * 2 + M * K + M * (K // 128) * 4
+    aq_gbs = aq_bytes / (aq_ms * 1e-3) / 1e9
+    fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
+
+    out = {
+        "metric": METRIC, "value": round(tflops, 2), "unit": "TFLOPS", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3",
+        "data": "synthetic (seeded N(0,1) activations with 1% outlier channels x20, N(0,0.02) weights)",
+        "config": {"workload": "prefill-shaped linear: act_quant + block-scaled FP8 GEMM, "
+                               "M=4096 N=28672 K=8192, 128-ch act groups, 128x128 weight blocks, fp32 scales, "
+                               "bf16 out", "M_per_gpu": M, "N": N, "K": K, "parallelism": f"dp{world} (token batches)",
+                   "l2": "inputs larger than L2 (W 235 MB); no flush"},
+        "gpu_launches": 2 * args.steps,
+        "e2e": {"value": round(e2e_tflops, 2), "unit": "TFLOPS", "h2d_bytes_per_step": M * K * 2,
+                "d2h_bytes_per_step": M * N * 2},
+        "roofline": {"bound": "tensor", "kernel": "k_gemm_wide", "achieved": round(gemm_tflops, 1),
+                     "peak": round(fp8_peak, 1), "unit": "TFLOP/s", "frac": round(gemm_tflops / fp8_peak, 4),
+                     "peak_source": f"{peak_src} bf16 burst x {FP8_OVER_BF16} (nominal fp8/bf16 ratio)",
+                     "traffic": profiled_traffic("k_gemm_wide prefill")},
+        "act_quant": {"GB/s": round(aq_gbs, 1), "us": round(aq_ms * 1e3, 2), "bytes": aq_bytes,
+                      "peak_GB/s": peaks["hbm_gbs"], "frac": round(aq_gbs / peaks["hbm_gbs"], 4),
+                      "bound": "hbm", "peak_source": peak_src,
+                      "traffic": profiled_traffic("k_act_quant prefill")},
+        "gemm_us": round(gm_ms * 1e3, 2),
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_rows:
+        out["rows"] = measure_rows(dev, peaks)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline_prefill(S)
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def time_launches(fn, iters, warm=2):
+    import torch
+    for _ in range(warm):
+        fn()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record()
+    for _ in range(iters):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / iters
+
+
+def measure_rows(dev, peaks):
+    """Every hot-path row on its own configuration (CUDA events, a few launches each)."""
+    import torch
+    import fp8_block_scaled_12_b200 as F
+    import synth
+    res = {}
+    hbm = peaks["hbm_gbs"]
+    fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
+    # act_quant sweep (per-128 fp32 and ue8m0) and per-tensor e4m3 / e5m2 at 16384 x 7168
+    x = synth.activations(16384, 7168, seed=0, dist="t3", device=dev)
+    M, K = x.shape
+    q = torch.empty((M, K), dtype=torch.uint8, device=dev)
+    s = torch.empty((M, K // 128), dtype=torch.float32, device=dev)
+    s1 = torch.empty((1,), dtype=torch.float32, device=dev)
+    for name, sf in (("act_quant_fp32", F.SCALE_FP32), ("act_quant_ue8m0", F.SCALE_UE8M0)):
+        ms = time_launches(lambda: F.fp8_act_quant(x, q, s, scale_fmt=sf), 20)
+        b = M * K * 3 + M * (K // 128) * 4
+        res[name + " 16384x7168"] = {"GB/s": round(b / ms / 1e6, 1), "frac_hbm": round(b / ms / 1e6 / hbm, 4)}
+    for name, fmt in (("per_tensor_e4m3", F.E4M3), ("per_tensor_e5m2", F.E5M2)):
+        ms = time_launches(lambda: F.fp8_weight_quant(x, q, s1, block=0, fmt=fmt), 10)
+        b = M * K * 3 + 4
+        res[name + " 16384x7168"] = {"GB/s (algorithmic 3 B/elt)": round(b / ms / 1e6, 1),
+                                      "frac_hbm": round(b / ms / 1e6 / hbm, 4)}
+    del x, q, s
+    # weight_quant 128x128 on the prefill weight
+    w = synth.weights(28672, 8192, 0.02, seed=0, device=dev)
+    qw = torch.empty(w.shape, dtype=torch.uint8, device=dev)
+    sw = torch.empty((224, 64), dtype=torch.float32, device=dev)
+    ms = time_launches(lambda: F.fp8_weight_quant(w, qw, sw), 10)
+    b = w.numel() * 3 + sw.numel() * 4
+    res["weight_quant 28672x8192"] = {"GB/s": round(b / ms / 1e6, 1), "frac_hbm": round(b / ms / 1e6 / hbm, 4)}
+    del w, qw, sw
+    # decode GEMM, ue8m0, M in {1, 8, 32, 64}
+    wd = synth.weights(18432, 7168, 0.015, seed=0, device=dev)
+    qwd, swd = F.weight_quant(wd, scale_fmt=F.SCALE_UE8M0)
+    del wd
+    for Md in (1, 8, 32, 64):
+        xd = synth.activations(Md, 7168, seed=0, device=dev)
+        qa, sa = F.act_quant(xd, scale_fmt=F.SCALE_UE8M0)
+        y = torch.empty((Md, 18432), dtype=torch.bfloat16, device=dev)
+        ms = time_launches(lambda: F.fp8_block_gemm(qa, sa, qwd, swd, y), 20)
+        b = 18432 * 7168 + swd.numel() * 4 + Md * (7168 + 56 * 4 + 18432 * 2)
+        res[f"decode_gemm M={Md}"] = {"us": round(ms * 1e3, 2), "GB/s": round(b / ms / 1e6, 1),
+                                      "frac_hbm": round(b / ms / 1e6 / hbm, 4),
+                                      "TFLOPS": round(2 * Md * 18432 * 7168 / ms / 1e9, 2)}
+    del qwd, swd
+    # grouped MoE GEMM
+    p = synth.MOE.params
+    row_token, _, off = synth.routing(p["T"], p["E"], p["topk"], seed=0)
+    xt = synth.activations(p["T"], p["K"], seed=0, device=dev)
+    qa, sa = F.act_quant(xt[row_token.to(dev)])
+    E, N, K = p["E"], p["N"], p["K"]
+    qwe = torch.empty((E, N, K), dtype=torch.uint8, device=dev)
+    swe = torch.empty((E, N // 128, K // 128), dtype=torch.float32, device=dev)
+    for e in range(E):
+        F.fp8_weight_quant(synth.weights(N, K, p["w_std"], seed=0, chunk=e, device=dev), qwe[e], swe[e])
+    y = torch.empty((qa.shape[0], N), dtype=torch.bfloat16, device=dev)
+    offd = off.to(dev)
+    ms = time_launches(lambda: F.fp8_grouped_gemm(qa, sa, qwe, swe, offd, y), 5)
+    fl = 2.0 * qa.shape[0] * N * K
+    b = qwe.numel() + swe.numel() * 4 + qa.numel() + sa.numel() * 4 + y.numel() * 2
+    res["grouped_gemm moe 32768x2048x7168 E=256"] = {"us": round(ms * 1e3, 1),
+                                                    "TFLOPS": round(fl / ms / 1e9, 1),
+                                                    "frac_fp8_peak": round(fl / ms / 1e9 / fp8_peak, 4),
+                                                    "GB/s": round(b / ms / 1e6, 1),
+                                                    "frac_hbm": round(b / ms / 1e6 / hbm, 4)}
+    assert F.fp8_device_error() == 0
+    return res
+
+
+def cpu_baseline_prefill(S):
+    """The oracle as it stands, single-threaded, on a bounded sample of the prefill
+    workload: act_quant of 2 rows and the fp64 GEMM of 1 row x 4096 columns."""
+    import oracle as O
+    K = S["K"]
+    x = S["x"][:2].cpu()
+    t = time.perf_counter()
+    qa, sa = O.act_quant(x)
+    t_aq = time.perf_counter() - t
+    qw = S["qw"][:4096].cpu().numpy()
+    sw = S["sw"][:32].cpu().numpy()
+    t = time.perf_counter()
+    O.gemm_rows(qa[:1], sa[:1], qw, sw)
+    t_g = time.perf_counter() - t
+    fl = 2.0 * 1 * 4096 * K
+    return {"value": round(fl / (t_aq / 2 + t_g) / 1e12, 6), "unit": "TFLOPS", "cores": 1, "kind": "oracle",
+            "sample": "act_quant of 1 row (timed on 2) + fp64 GEMM of 1 row x 4096 cols x 8192 of the "
+                      "prefill workload, single thread",
+            "seconds": round(t_aq + t_g, 2)}
+
+
+def run_other(args, world, rank, dev, peaks, peak_src):
+    """Secondary workloads: one JSON line each (not the headline)."""
+    import torch
+    out = {"metric": METRIC, "workload": args.workload, "n_gpus": world}
+    out["rows"] = measure_rows(dev, peaks)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+# ------------------------------------------------------------- reference arm
+def run_reference(args, world, rank):
+    """The CPU oracle on the prefill workload's shapes: each step is a bounded sample
+    (act_quant of one row and the fp64 GEMM of that row against 1024 weight rows)."""
+    if rank != 0:
+        return
+    import oracle as O
+    import synth
+    p = synth.PREFILL.params
+    K = p["K"]
+    ch = synth.outlier_channels(K, synth.n_outliers(K, p["outlier_frac"]), seed=0)
+    x = synth.activations(4, K, seed=0, outliers=ch, factor=p["factor"])
+    w = synth.weights(1024, K, p["w_std"], seed=0)
+    qw, sw = O.weight_quant(w)
+    n = 1024
+
+    def step():
+        qa, sa = O.act_quant(x[:1])
+        O.gemm_rows(qa, sa, qw, sw)
+
+    for _ in range(args.warmup):
+        step()
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t
+    fl = 2.0 * n * K * args.steps
+    v = fl / dt / 1e12
+    out = {"impl": "reference", "metric": METRIC, "value": round(v, 6), "unit": "TFLOPS", "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3 / args.steps, 2),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic", "config": {"workload": "prefill-shaped linear (bounded sample: 1 row x 1024 "
+                                                       "weight rows x 8192 per step)"},
+           "cpu_baseline": {"value": round(v, 6), "unit": "TFLOPS", "cores": 1, "kind": "oracle",
+                            "sample": "act_quant of 1 row + fp64 GEMM of 1 row x 1024 x 8192 per step"},
+           "e2e": {"value": round(v, 6), "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["prefill", "decode", "moe", "sweep"], default="prefill")
+    ap.add_argument("--no-rows", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+    run_ours(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,187 @@
+"""B200-native FP8 W8A8 linear layer -- Python binding of libfp8lin.so.
+
+The binding only marshals arguments: it passes device pointers, shapes and the
+current CUDA stream to the C ABI declared in include/fp8lin.h, where every step
+of the path runs in hand-written sm_100a kernels.  PyTorch supplies device memory
+and streams.  There is no fallback: importing this package fails if the CUDA
+library has not been built, and every call raises Fp8Error on a non-zero status.
+
+Functions with the C names (``fp8_act_quant``, ``fp8_weight_quant``,
+``fp8_block_gemm``, ``fp8_grouped_gemm``) take preallocated output tensors; the
+short names (``act_quant``, ``weight_quant``, ``block_gemm``, ``grouped_gemm``)
+allocate the outputs with torch and call them.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "E4M3", "E5M2", "SCALE_FP32", "SCALE_UE8M0", "OUT_BF16", "OUT_FP32", "Fp8Error", "LIB_PATH",
+    "fp8_act_quant", "fp8_weight_quant", "fp8_block_gemm", "fp8_grouped_gemm",
+    "fp8_status_string", "fp8_device_error",
+    "act_quant", "weight_quant", "block_gemm", "grouped_gemm", "EXPORTS",
+]
+
+E4M3, E5M2 = 0, 1
+SCALE_FP32, SCALE_UE8M0 = 0, 1
+OUT_BF16, OUT_FP32 = 0, 1
+FP8_OK = 0
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfp8lin.so")
+EXPORTS = ("fp8_act_quant", "fp8_weight_quant", "fp8_block_gemm", "fp8_grouped_gemm",
+           "fp8_status_string", "fp8_device_error")
+
+
+class Fp8Error(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} failed: {code} ({fp8_status_string(code)})")
+        self.code = code
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing; build it with `python -m fp8_block_scaled_12_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i64, ci = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    L.fp8_act_quant.argtypes = [vp, i64, i64, i64, ci, ci, ci, vp, vp, vp]
+    L.fp8_weight_quant.argtypes = [vp, i64, i64, ci, ci, ci, vp, vp, vp]
+    L.fp8_block_gemm.argtypes = [vp, vp, vp, vp, i64, i64, i64, ci, vp, vp]
+    L.fp8_grouped_gemm.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, ci, vp, vp]
+    L.fp8_status_string.argtypes = [ci]
+    L.fp8_status_string.restype = ctypes.c_char_p
+    L.fp8_device_error.argtypes = [vp]
+    for name in ("fp8_act_quant", "fp8_weight_quant", "fp8_block_gemm", "fp8_grouped_gemm", "fp8_device_error"):
+        getattr(L, name).restype = ci
+    return L
+
+
+lib = _load()
+
+
+def fp8_status_string(code: int) -> str:
+    return lib.fp8_status_string(int(code)).decode()
+
+
+def _check(fn: str, code: int) -> None:
+    if code != FP8_OK:
+        raise Fp8Error(fn, code)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("fp8 library tensors must live on a CUDA device")
+    return t.data_ptr()
+
+
+def _u8(t: torch.Tensor) -> torch.Tensor:
+    if t.dtype in (torch.float8_e4m3fn, torch.float8_e5m2):
+        return t.view(torch.uint8)
+    if t.dtype != torch.uint8:
+        raise TypeError(f"FP8 codes must be uint8 / float8, got {t.dtype}")
+    return t
+
+
+# ------------------------------------------------------------- C names
+def fp8_act_quant(x: torch.Tensor, q: torch.Tensor, s: torch.Tensor, group: int = 128, fmt: int = E4M3,
+                  scale_fmt: int = SCALE_FP32, stream=None) -> None:
+    """Per-token, per-group quantisation of bf16 x [M, K] (row stride x.stride(0)) into
+    codes q [M, K] and fp32 scales s [M, ceil(K/group)]."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    assert q.is_contiguous() and s.is_contiguous() and s.dtype == torch.float32
+    M, K = x.shape
+    _check("fp8_act_quant", lib.fp8_act_quant(_ptr(x), M, K, x.stride(0), group, fmt, scale_fmt,
+                                              _ptr(_u8(q)), _ptr(s), _stream(stream)))
+
+
+def fp8_weight_quant(w: torch.Tensor, q: torch.Tensor, s_inv: torch.Tensor, block: int = 128,
+                     fmt: int = E4M3, scale_fmt: int = SCALE_FP32, stream=None) -> None:
+    """128x128-block (block=128) or per-tensor (block=0) quantisation of bf16 w [N, K]."""
+    assert w.dtype == torch.bfloat16 and w.is_contiguous()
+    assert q.is_contiguous() and s_inv.is_contiguous() and s_inv.dtype == torch.float32
+    w2 = w.reshape(-1, w.shape[-1])
+    N, K = w2.shape
+    _check("fp8_weight_quant", lib.fp8_weight_quant(_ptr(w2), N, K, block, fmt, scale_fmt, _ptr(_u8(q)),
+                                                    _ptr(s_inv), _stream(stream)))
+
+
+def _out_code(y: torch.Tensor) -> int:
+    if y.dtype == torch.bfloat16:
+        return OUT_BF16
+    if y.dtype == torch.float32:
+        return OUT_FP32
+    raise TypeError(f"output must be bf16 or fp32, got {y.dtype}")
+
+
+def fp8_block_gemm(qa: torch.Tensor, sa: torch.Tensor, qw: torch.Tensor, sw: torch.Tensor, y: torch.Tensor,
+                   stream=None) -> None:
+    """y [M, N] = block-scaled FP8 GEMM of codes qa [M, K] (scales sa [M, K/128]) and
+    qw [N, K] (scales sw [ceil(N/128), K/128])."""
+    for t in (qa, sa, qw, sw, y):
+        assert t.is_contiguous()
+    M, K = qa.shape
+    N = qw.shape[0]
+    _check("fp8_block_gemm", lib.fp8_block_gemm(_ptr(_u8(qa)), _ptr(sa), _ptr(_u8(qw)), _ptr(sw), M, N, K,
+                                                _out_code(y), _ptr(y), _stream(stream)))
+
+
+def fp8_grouped_gemm(qa: torch.Tensor, sa: torch.Tensor, qw: torch.Tensor, sw: torch.Tensor,
+                     offsets: torch.Tensor, y: torch.Tensor, stream=None) -> None:
+    """Grouped GEMM over expert-sorted rows: qw [E, N, K], sw [E, ceil(N/128), K/128],
+    offsets device int32 [E+1]."""
+    for t in (qa, sa, qw, sw, offsets, y):
+        assert t.is_contiguous()
+    assert offsets.dtype == torch.int32
+    total_M, K = qa.shape
+    E, N, _ = qw.shape
+    _check("fp8_grouped_gemm", lib.fp8_grouped_gemm(_ptr(_u8(qa)), _ptr(sa), _ptr(_u8(qw)), _ptr(sw),
+                                                    _ptr(offsets), E, total_M, N, K, _out_code(y), _ptr(y),
+                                                    _stream(stream)))
+
+
+def fp8_device_error(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device-side wait status."""
+    return int(lib.fp8_device_error(_stream(stream)))
+
+
+# ------------------------------------------------- allocating wrappers
+def act_quant(x: torch.Tensor, group: int = 128, fmt: int = E4M3, scale_fmt: int = SCALE_FP32, stream=None):
+    M, K = x.shape
+    q = torch.empty((M, K), dtype=torch.uint8, device=x.device)
+    s = torch.empty((M, (K + group - 1) // group), dtype=torch.float32, device=x.device)
+    fp8_act_quant(x, q, s, group, fmt, scale_fmt, stream)
+    return q, s
+
+
+def weight_quant(w: torch.Tensor, block: int = 128, fmt: int = E4M3, scale_fmt: int = SCALE_FP32,
+                 stream=None):
+    N, K = w.shape
+    q = torch.empty((N, K), dtype=torch.uint8, device=w.device)
+    shape = (1,) if block == 0 else ((N + block - 1) // block, (K + block - 1) // block)
+    s = torch.empty(shape, dtype=torch.float32, device=w.device)
+    fp8_weight_quant(w, q, s, block, fmt, scale_fmt, stream)
+    return q, s
+
+
+def block_gemm(qa, sa, qw, sw, out_dtype=torch.bfloat16, stream=None):
+    y = torch.empty((qa.shape[0], qw.shape[0]), dtype=out_dtype, device=qa.device)
+    fp8_block_gemm(qa, sa, qw, sw, y, stream)
+    return y
+
+
+def grouped_gemm(qa, sa, qw, sw, offsets, out_dtype=torch.bfloat16, stream=None):
+    y = torch.empty((qa.shape[0], qw.shape[1]), dtype=out_dtype, device=qa.device)
+    fp8_grouped_gemm(qa, sa, qw, sw, offsets, y, stream)
+    return y

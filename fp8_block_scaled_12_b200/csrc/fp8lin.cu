@@ -1,0 +1,274 @@
+// fp8lin.cu -- the C ABI (include/fp8lin.h): argument checks, TMA descriptors and
+// kernel launches.  The whole library is this one translation unit.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/fp8lin.h"
+#include "gemm.cuh"
+#include "ptx.cuh"
+#include "quant.cuh"
+
+using namespace fp8lin;
+
+namespace {
+
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+inline int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return FP8_OK;
+  return FP8_ERR_CUDA;
+}
+
+// Streaming multiprocessors of the current device (cached per device).
+int num_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+// ---------------------------------------------------------------- TMA maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D map over a row-major byte matrix [rows][cols] (row stride = cols bytes),
+// box = box_rows x 128 bytes, 128-byte swizzle, out-of-range reads give zeros.
+bool make_map_u8(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t box[2] = {128, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------- GEMM launches
+constexpr int kWideStages = 4;
+
+// The warpgroup register split inside the GEMM kernels (setmaxnreg) draws on the
+// registers the CTA was launched with; refuse to launch a build whose register
+// count differs from the one the split was sized for (it could never satisfy
+// the increase).
+template <typename K>
+bool launch_regs_ok(K kern) {
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return false;
+  return fa.numRegs == int(kLaunchRegs);
+}
+
+template <int NT, int STAGES>
+int launch_swap(const void* qa, const void* qw, const GemmArgs& a, int64_t w_rows, cudaStream_t st) {
+  using C = SwapCfg<NT, STAGES>;
+  CUtensorMap mw, mx;
+  if (!make_map_u8(&mw, qw, uint64_t(w_rows), uint64_t(a.K), 128)) return FP8_ERR_CUDA;
+  if (!make_map_u8(&mx, qa, uint64_t(a.M > 0 ? a.M : 1), uint64_t(a.K), 32)) return FP8_ERR_CUDA;
+  auto kern = k_gemm_swap<NT, STAGES>;
+  if (!launch_regs_ok(kern)) return FP8_ERR_UNSUPPORTED;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(C::SMEM));
+  if (e != cudaSuccess) return FP8_ERR_CUDA;
+  const int nbn = (a.N + 127) / 128;
+  const int64_t units = int64_t(a.E) * nbn;
+  const int grid = int(units < num_sms() ? units : num_sms());
+  kern<<<grid, kThreads, C::SMEM, st>>>(mw, mx, a);
+  return cuda_status(cudaGetLastError());
+}
+
+int launch_wide(const void* qa, const void* qw, const GemmArgs& a, cudaStream_t st) {
+  using C = WideCfg<kWideStages>;
+  CUtensorMap ma, mb;
+  if (!make_map_u8(&ma, qa, uint64_t(a.M), uint64_t(a.K), C::BM)) return FP8_ERR_CUDA;
+  if (!make_map_u8(&mb, qw, uint64_t(a.N), uint64_t(a.K), C::BN)) return FP8_ERR_CUDA;
+  auto kern = k_gemm_wide<kWideStages>;
+  if (!launch_regs_ok(kern)) return FP8_ERR_UNSUPPORTED;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(C::SMEM));
+  if (e != cudaSuccess) return FP8_ERR_CUDA;
+  const int64_t tiles = int64_t((a.M + C::BM - 1) / C::BM) * ((a.N + C::BN - 1) / C::BN);
+  const int grid = int(tiles < num_sms() ? tiles : num_sms());
+  kern<<<grid, kThreads, C::SMEM, st>>>(ma, mb, a);
+  return cuda_status(cudaGetLastError());
+}
+
+// ------------------------------------------------------ quantiser launches
+template <int FMT, int SF>
+int launch_act_quant(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q, float* s,
+                     cudaStream_t st) {
+  constexpr int U = 4;
+  const int64_t ng = (K + 127) / 128;
+  const int64_t items = M * ng;
+  const int64_t per_block = (256 / 32) * 2 * U;
+  int64_t blocks = (items + per_block - 1) / per_block;
+  const int64_t cap = int64_t(num_sms()) * 8;
+  if (blocks > cap) blocks = cap;
+  k_act_quant<FMT, SF, U><<<int(blocks), 256, 0, st>>>(x, M, K, ldx, q, s);
+  return cuda_status(cudaGetLastError());
+}
+
+template <int FMT, int SF>
+int launch_block_quant(const uint16_t* w, int64_t N, int64_t K, uint8_t* q, float* s, cudaStream_t st) {
+  dim3 grid(unsigned((K + 127) / 128), unsigned((N + 127) / 128));
+  k_block_quant<FMT, SF><<<grid, 256, 0, st>>>(w, N, K, q, s);
+  return cuda_status(cudaGetLastError());
+}
+
+template <int FMT, int SF>
+int launch_tensor_quant(const uint16_t* x, int64_t n, uint8_t* q, float* s, cudaStream_t st) {
+  const int64_t n8 = n / 8;
+  int64_t blocks = (n8 + 255) / 256;
+  const int64_t cap = int64_t(num_sms()) * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  unsigned int* slot = reinterpret_cast<unsigned int*>(s);
+  cudaError_t e = cudaMemsetAsync(slot, 0, sizeof(unsigned int), st);
+  if (e != cudaSuccess) return FP8_ERR_CUDA;
+  k_tensor_amax<<<int(blocks), 256, 0, st>>>(x, n8, slot);
+  k_tensor_cast<FMT, SF><<<int(blocks), 256, 0, st>>>(x, n8, slot, q);
+  k_tensor_scale<FMT, SF><<<1, 1, 0, st>>>(slot);
+  return cuda_status(cudaGetLastError());
+}
+
+}  // namespace
+
+// =====================================================================
+// C ABI
+// =====================================================================
+extern "C" {
+
+const char* fp8_status_string(int status) {
+  switch (status) {
+    case FP8_OK: return "ok";
+    case FP8_ERR_INVALID_ARG: return "invalid argument";
+    case FP8_ERR_SHAPE: return "unsupported shape";
+    case FP8_ERR_ALIGNMENT: return "misaligned pointer or leading dimension";
+    case FP8_ERR_UNSUPPORTED: return "unsupported option";
+    case FP8_ERR_CUDA: return "CUDA error";
+    case FP8_ERR_TIMEOUT: return "device wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int fp8_act_quant(const void* x, int64_t M, int64_t K, int64_t ldx, int group, int fmt, int scale_fmt,
+                  void* q, float* s, void* stream) {
+  if (M < 0 || K <= 0 || ldx < K) return FP8_ERR_INVALID_ARG;
+  if (fmt != FP8_E4M3 && fmt != FP8_E5M2) return FP8_ERR_INVALID_ARG;
+  if (scale_fmt != FP8_SCALE_FP32 && scale_fmt != FP8_SCALE_UE8M0) return FP8_ERR_INVALID_ARG;
+  if (group != 128) return FP8_ERR_UNSUPPORTED;
+  if (K % 16 != 0) return FP8_ERR_SHAPE;
+  if (M == 0) return FP8_OK;
+  if (!x || !q || !s) return FP8_ERR_INVALID_ARG;
+  if (ldx % 8 != 0 || !aligned(x, 16) || !aligned(q, 16) || !aligned(s, 4)) return FP8_ERR_ALIGNMENT;
+  const uint16_t* xb = static_cast<const uint16_t*>(x);
+  uint8_t* qb = static_cast<uint8_t*>(q);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (fmt == FP8_E4M3)
+    return scale_fmt == FP8_SCALE_FP32 ? launch_act_quant<kE4M3, kScaleFp32>(xb, M, K, ldx, qb, s, st)
+                                       : launch_act_quant<kE4M3, kScaleUe8m0>(xb, M, K, ldx, qb, s, st);
+  return scale_fmt == FP8_SCALE_FP32 ? launch_act_quant<kE5M2, kScaleFp32>(xb, M, K, ldx, qb, s, st)
+                                     : launch_act_quant<kE5M2, kScaleUe8m0>(xb, M, K, ldx, qb, s, st);
+}
+
+int fp8_weight_quant(const void* w, int64_t N, int64_t K, int block, int fmt, int scale_fmt, void* q,
+                     float* s_inv, void* stream) {
+  if (N < 0 || K <= 0) return FP8_ERR_INVALID_ARG;
+  if (fmt != FP8_E4M3 && fmt != FP8_E5M2) return FP8_ERR_INVALID_ARG;
+  if (scale_fmt != FP8_SCALE_FP32 && scale_fmt != FP8_SCALE_UE8M0) return FP8_ERR_INVALID_ARG;
+  if (block != 128 && block != 0) return FP8_ERR_UNSUPPORTED;
+  if (K % 16 != 0) return FP8_ERR_SHAPE;
+  if (N == 0) return FP8_OK;
+  if (!w || !q || !s_inv) return FP8_ERR_INVALID_ARG;
+  if (!aligned(w, 16) || !aligned(q, 16) || !aligned(s_inv, 4)) return FP8_ERR_ALIGNMENT;
+  const uint16_t* wb = static_cast<const uint16_t*>(w);
+  uint8_t* qb = static_cast<uint8_t*>(q);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (block == 128) {
+    if (fmt == FP8_E4M3)
+      return scale_fmt == FP8_SCALE_FP32 ? launch_block_quant<kE4M3, kScaleFp32>(wb, N, K, qb, s_inv, st)
+                                         : launch_block_quant<kE4M3, kScaleUe8m0>(wb, N, K, qb, s_inv, st);
+    return scale_fmt == FP8_SCALE_FP32 ? launch_block_quant<kE5M2, kScaleFp32>(wb, N, K, qb, s_inv, st)
+                                       : launch_block_quant<kE5M2, kScaleUe8m0>(wb, N, K, qb, s_inv, st);
+  }
+  const int64_t n = N * K;
+  if (fmt == FP8_E4M3)
+    return scale_fmt == FP8_SCALE_FP32 ? launch_tensor_quant<kE4M3, kScaleFp32>(wb, n, qb, s_inv, st)
+                                       : launch_tensor_quant<kE4M3, kScaleUe8m0>(wb, n, qb, s_inv, st);
+  return scale_fmt == FP8_SCALE_FP32 ? launch_tensor_quant<kE5M2, kScaleFp32>(wb, n, qb, s_inv, st)
+                                     : launch_tensor_quant<kE5M2, kScaleUe8m0>(wb, n, qb, s_inv, st);
+}
+
+static int check_gemm_common(const void* qa, const float* sa, const void* qw, const float* sw, int64_t M,
+                             int64_t N, int64_t K, int out_dtype, void* y) {
+  if (M < 0 || N <= 0 || K <= 0) return FP8_ERR_INVALID_ARG;
+  if (out_dtype != FP8_OUT_BF16 && out_dtype != FP8_OUT_FP32) return FP8_ERR_INVALID_ARG;
+  if (K % 128 != 0 || N % 16 != 0) return FP8_ERR_SHAPE;
+  if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return FP8_ERR_SHAPE;
+  if (!qw || !sw) return FP8_ERR_INVALID_ARG;
+  if (M > 0 && (!qa || !sa || !y)) return FP8_ERR_INVALID_ARG;
+  if (!aligned(qw, 16) || !aligned(sw, 4)) return FP8_ERR_ALIGNMENT;
+  if (M > 0 && (!aligned(qa, 16) || !aligned(sa, 4) || !aligned(y, 16))) return FP8_ERR_ALIGNMENT;
+  return FP8_OK;
+}
+
+int fp8_block_gemm(const void* qa, const float* sa, const void* qw, const float* sw, int64_t M, int64_t N,
+                   int64_t K, int out_dtype, void* y, void* stream) {
+  int rc = check_gemm_common(qa, sa, qw, sw, M, N, K, out_dtype, y);
+  if (rc != FP8_OK) return rc;
+  if (M == 0) return FP8_OK;
+  GemmArgs a{sa, sw, y, nullptr, int(M), int(N), int(K), 1, out_dtype == FP8_OUT_FP32 ? 1 : 0};
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (M <= 64) return launch_swap<64, 8>(qa, qw, a, N, st);
+  if (M <= 128) return launch_swap<128, 6>(qa, qw, a, N, st);
+  if (M <= 256) return launch_swap<256, 4>(qa, qw, a, N, st);
+  return launch_wide(qa, qw, a, st);
+}
+
+int fp8_grouped_gemm(const void* qa, const float* sa, const void* qw, const float* sw,
+                     const int32_t* group_offsets, int64_t E, int64_t total_M, int64_t N, int64_t K,
+                     int out_dtype, void* y, void* stream) {
+  int rc = check_gemm_common(qa, sa, qw, sw, total_M, N, K, out_dtype, y);
+  if (rc != FP8_OK) return rc;
+  if (E <= 0 || E > INT32_MAX || !group_offsets) return FP8_ERR_INVALID_ARG;
+  if (!aligned(group_offsets, 4)) return FP8_ERR_ALIGNMENT;
+  if (E * N > INT32_MAX) return FP8_ERR_SHAPE;
+  if (total_M == 0) return FP8_OK;
+  GemmArgs a{sa, sw, y, group_offsets, int(total_M), int(N), int(K), int(E),
+             out_dtype == FP8_OUT_FP32 ? 1 : 0};
+  return launch_swap<256, 4>(qa, qw, a, E * N, static_cast<cudaStream_t>(stream));
+}
+
+int fp8_device_error(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return FP8_ERR_CUDA;
+  unsigned int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v)) != cudaSuccess) return FP8_ERR_CUDA;
+  if (v != 0 && cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess) return FP8_ERR_CUDA;
+  return v ? FP8_ERR_TIMEOUT : FP8_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,498 @@
+// gemm.cuh -- block-scaled FP8 GEMMs on the 5th-generation tensor cores (sm_100a).
+//
+// Operation ("FP8 推理提速 83.6%: DeepSeek-V3 在 AMD MI250 上的完整落地指南", 运行时:
+// fp8_gemm(x, scale, weight, weight.scale); "LLM 推理的 FP8 混合精度工程 2026",
+// section 3: FP8 products, FP32 accumulation):
+//
+//   y[m][n] = sum_kb sa[m][kb] * sw[n/128][kb] * P_kb[m][n],
+//   P_kb[m][n] = sum_{k in K-block kb} qa[m][k] * qw[n][k]   (E4M3 x E4M3 -> fp32)
+//
+// Both kernels share one pipeline, warp-specialised inside a 384-thread CTA:
+//   warp 0        TMA producer: one lane streams 128-deep K-blocks of both operands
+//                 into a ring of shared-memory stages (128-byte swizzle, K-major).
+//   warp 1        MMA issuer: one lane issues 4 x tcgen05.mma (K = 32 each) per
+//                 K-block into one of two tensor-memory partial buffers, then
+//                 commits to the stage's "empty" barrier and the buffer's "full" one.
+//   warps 2-3     idle (their registers are handed to the epilogue).
+//   warps 4-11    promotion / epilogue, two warpgroups: per K-block each thread loads
+//                 its lane's partials from tensor memory (tcgen05.ld), frees the
+//                 buffer and folds them into fp32 register accumulators scaled by
+//                 sa * sw; after the last K-block it converts and stores the tile.
+// Because the running sum lives in registers, the MMA of K-block kb+1 overlaps the
+// promotion of K-block kb, and a CTA can start its next tile while it stores one.
+//
+//   k_gemm_wide   M-side = 128 activation rows, N-side = 256 weight rows per tile;
+//                 persistent over tiles, M fastest so concurrent CTAs share weights.
+//   k_gemm_swap   M-side = 128 weight rows, N-side = up to NT tokens: for decode
+//                 (few tokens) and for the grouped MoE GEMM, where the MMA's N is set
+//                 per tile to the expert's token count rounded up to 16.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "ptx.cuh"
+
+namespace fp8lin {
+
+constexpr int kBK = 128;                  // K-block = scale block = one 128-byte row
+constexpr int kThreads = 384;
+constexpr int kEpiThreads = 256;
+constexpr uint32_t kTileBytesPerRow = 128;
+// Register split between the producer/MMA warpgroup and the two epilogue
+// warpgroups.  The kernels are compiled for kLaunchRegs registers per thread
+// (launch bounds 384 x 1); the split must not exceed that pool:
+// 128 * kProducerRegs + 256 * kConsumerRegs == 384 * kLaunchRegs.
+constexpr uint32_t kLaunchRegs = 168;
+constexpr uint32_t kProducerRegs = 56;
+constexpr uint32_t kConsumerRegs = 224;
+static_assert(128 * kProducerRegs + 256 * kConsumerRegs <= 384 * kLaunchRegs, "register split exceeds pool");
+
+struct GemmArgs {
+  const float* sa;        // [rows][nkb]
+  const float* sw;        // [E][nbn][nkb]
+  void* y;                // [rows][N]
+  const int32_t* offsets; // grouped: device [E+1]; nullptr = one group [0, M)
+  int M;                  // activation rows (total rows for grouped)
+  int N;                  // weight rows per expert
+  int K;
+  int E;
+  int out_fp32;
+};
+
+// Shared-memory bookkeeping placed after the stage buffers.
+template <int STAGES>
+struct alignas(8) PipeState {
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t csfull[2][2];   // swap kernel: column-scale slot handoff, [warpgroup][slot]
+  uint32_t tmem_base;
+  int abort;
+};
+
+// Store 8 consecutive outputs (bf16 or fp32) for one row.
+__device__ __forceinline__ void store8(void* y, bool fp32, int64_t idx, const float* v) {
+  if (fp32) {
+    float4* p = reinterpret_cast<float4*>(reinterpret_cast<float*>(y) + idx);
+    p[0] = make_float4(v[0], v[1], v[2], v[3]);
+    p[1] = make_float4(v[4], v[5], v[6], v[7]);
+  } else {
+    uint4 o;
+    __nv_bfloat162 b0 = __floats2bfloat162_rn(v[0], v[1]);
+    __nv_bfloat162 b1 = __floats2bfloat162_rn(v[2], v[3]);
+    __nv_bfloat162 b2 = __floats2bfloat162_rn(v[4], v[5]);
+    __nv_bfloat162 b3 = __floats2bfloat162_rn(v[6], v[7]);
+    o.x = *reinterpret_cast<uint32_t*>(&b0);
+    o.y = *reinterpret_cast<uint32_t*>(&b1);
+    o.z = *reinterpret_cast<uint32_t*>(&b2);
+    o.w = *reinterpret_cast<uint32_t*>(&b3);
+    *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(y) + idx) = o;
+  }
+}
+
+// =====================================================================
+// Wide kernel: tile = 128 activation rows x 256 weight rows.
+// =====================================================================
+template <int STAGES>
+struct WideCfg {
+  static constexpr int BM = 128, BN = 256;
+  static constexpr uint32_t A_BYTES = BM * kTileBytesPerRow;       // 16 KB
+  static constexpr uint32_t B_BYTES = BN * kTileBytesPerRow;       // 32 KB
+  static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr uint32_t TMEM_COLS = 2 * BN;                    // 512
+  static constexpr size_t SMEM = 1024 + size_t(STAGES) * STAGE_BYTES + sizeof(PipeState<STAGES>);
+};
+
+template <int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_gemm_wide(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const GemmArgs args) {
+  using C = WideCfg<STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  PipeState<STAGES>* ps = reinterpret_cast<PipeState<STAGES>*>(gbase + size_t(STAGES) * C::STAGE_BYTES);
+  volatile int* abort = &ps->abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int num_m = (args.M + C::BM - 1) / C::BM;
+  const int num_n = (args.N + C::BN - 1) / C::BN;
+  const int num_tiles = num_m * num_n;
+  const int nkb = args.K / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(&ps->full[s]), 1);
+      mbar_init(smem_u32(&ps->empty[s]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&ps->tfull[b]), 1);
+      mbar_init(smem_u32(&ps->tempty[b]), kEpiThreads / 32);
+    }
+    ps->abort = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&ps->tmem_base), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ps->tmem_base;
+
+  if (warp < 4) {
+    setmaxnreg_dec<kProducerRegs>();
+    if (warp == 0 && lane == 0) {
+      // ------------------------------------------------ TMA producer
+      uint32_t it = 0;
+      for (int tile = blockIdx.x; tile < num_tiles && !*abort; tile += gridDim.x) {
+        const int mb = tile % num_m, nb = tile / num_m;
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1u;
+          if (!mbar_wait(smem_u32(&ps->empty[s]), ph ^ 1u, abort)) break;
+          const uint32_t sa_ = base + s * C::STAGE_BYTES;
+          const uint32_t bar = smem_u32(&ps->full[s]);
+          mbar_arrive_expect_tx(bar, C::STAGE_BYTES);
+          tma_load_2d(sa_, &tmA, bar, kb * kBK, mb * C::BM);
+          tma_load_2d(sa_ + C::A_BYTES, &tmB, bar, kb * kBK, nb * C::BN);
+        }
+      }
+    } else if (warp == 1 && lane == 0) {
+      // ------------------------------------------------ MMA issuer
+      constexpr uint32_t idesc = idesc_f8_e4m3_f32(C::BM, C::BN);
+      uint32_t it = 0, kbc = 0;
+      for (int tile = blockIdx.x; tile < num_tiles && !*abort; tile += gridDim.x) {
+        for (int kb = 0; kb < nkb; ++kb, ++it, ++kbc) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1u;
+          const uint32_t b = kbc & 1u;
+          const uint32_t tph = (kbc >> 1) & 1u;
+          if (!mbar_wait(smem_u32(&ps->tempty[b]), tph ^ 1u, abort)) break;
+          if (!mbar_wait(smem_u32(&ps->full[s]), ph, abort)) break;
+          tc_fence_after();
+          const uint32_t a_addr = base + s * C::STAGE_BYTES;
+          const uint32_t b_addr = a_addr + C::A_BYTES;
+          const uint32_t d = tmem + b * C::BN;
+#pragma unroll
+          for (int k = 0; k < kBK / 32; ++k)
+            mma_f8(d, sw128_kmajor_desc(a_addr + k * 32), sw128_kmajor_desc(b_addr + k * 32), idesc,
+                   k > 0 ? 1u : 0u);
+          mma_commit(smem_u32(&ps->empty[s]));
+          mma_commit(smem_u32(&ps->tfull[b]));
+        }
+      }
+    }
+  } else {
+    setmaxnreg_inc<kConsumerRegs>();
+    // ------------------------------------------------ promotion + epilogue
+    const int ew = warp - 4;             // 0..7
+    const int wg = ew >> 2;              // column half of the tile
+    const int quad = warp & 3;           // tensor-memory lane quadrant of this warp
+    const int row_in_tile = quad * 32 + lane;
+    const bool out32 = args.out_fp32 != 0;
+    uint32_t kbc = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      const int mb = tile % num_m, nb = tile / num_m;
+      const int64_t m = int64_t(mb) * C::BM + row_in_tile;
+      const int n0 = nb * C::BN + wg * 128;
+      const bool row_ok = m < args.M;
+      const bool cols_any = n0 < args.N;
+      const float* sa_row = args.sa + (row_ok ? m : 0) * nkb;
+      const float* sw_blk = args.sw + int64_t(cols_any ? n0 / 128 : 0) * nkb;
+      float acc[128];
+#pragma unroll
+      for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
+      float sa_next = row_ok ? __ldg(sa_row) : 0.0f;
+      float sw_next = cols_any ? __ldg(sw_blk) : 0.0f;
+      bool aborted = false;
+      for (int kb = 0; kb < nkb; ++kb, ++kbc) {
+        const float scale = sa_next * sw_next;
+        if (kb + 1 < nkb) {
+          sa_next = row_ok ? __ldg(sa_row + kb + 1) : 0.0f;
+          sw_next = cols_any ? __ldg(sw_blk + kb + 1) : 0.0f;
+        }
+        const uint32_t b = kbc & 1u;
+        if (!mbar_wait(smem_u32(&ps->tfull[b]), (kbc >> 1) & 1u, abort)) { aborted = true; break; }
+        tc_fence_after();
+        const uint32_t taddr = tmem + (uint32_t(quad * 32) << 16) + b * C::BN + wg * 128;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t p0[32], p1[32];
+          tmem_ld32(taddr + h * 64, p0);
+          tmem_ld32(taddr + h * 64 + 32, p1);
+          tmem_ld_wait();
+          if (h == 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&ps->tempty[b]));
+          }
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            acc[h * 64 + j] = fmaf(__uint_as_float(p0[j]), scale, acc[h * 64 + j]);
+            acc[h * 64 + 32 + j] = fmaf(__uint_as_float(p1[j]), scale, acc[h * 64 + 32 + j]);
+          }
+        }
+      }
+      if (aborted) break;
+      if (row_ok && cols_any) {
+#pragma unroll
+        for (int j = 0; j < 128; j += 8) {
+          if (n0 + j < args.N) store8(args.y, out32, m * args.N + n0 + j, &acc[j]);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (*abort) {
+    if (threadIdx.x == 0) settle_ns(200000);
+    __syncthreads();
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// =====================================================================
+// Swap kernel: tile = 128 weight rows x up to NT tokens (one expert's rows).
+// =====================================================================
+template <int NT, int STAGES>
+struct SwapCfg {
+  static constexpr uint32_t W_BYTES = 128 * kTileBytesPerRow;      // 16 KB
+  static constexpr uint32_t X_BYTES = NT * kTileBytesPerRow;
+  static constexpr uint32_t STAGE_BYTES = W_BYTES + X_BYTES;
+  static constexpr uint32_t TMEM_COLS = (2 * NT < 32) ? 32 : 2 * NT;
+  static constexpr int COLS_PER_WG = NT / 2;                       // token columns per warpgroup
+  static constexpr size_t CS_BYTES = 2 * NT * sizeof(float);   // [slot][NT] column scales
+  static constexpr size_t SMEM = 1024 + size_t(STAGES) * STAGE_BYTES + CS_BYTES + sizeof(PipeState<STAGES>);
+};
+
+// Unit u -> (expert, weight row-block); units of one expert are consecutive so the
+// expert's token rows are re-read from L2 while its weights stream from HBM once.
+__device__ __forceinline__ void group_range(const GemmArgs& a, int e, int& r0, int& r1) {
+  if (a.offsets == nullptr) {
+    r0 = 0;
+    r1 = a.M;
+  } else {
+    r0 = __ldg(a.offsets + e);
+    r1 = __ldg(a.offsets + e + 1);
+    r1 = min(r1, a.M);
+    r0 = min(r0, r1);
+  }
+}
+
+template <int NT, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_gemm_swap(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                const GemmArgs args) {
+  using C = SwapCfg<NT, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  float* colscale = reinterpret_cast<float*>(gbase + size_t(STAGES) * C::STAGE_BYTES);
+  PipeState<STAGES>* ps =
+      reinterpret_cast<PipeState<STAGES>*>(gbase + size_t(STAGES) * C::STAGE_BYTES + C::CS_BYTES);
+  volatile int* abort = &ps->abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nbn = (args.N + 127) / 128;
+  const int num_units = args.E * nbn;
+  const int nkb = args.K / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(&ps->full[s]), 1);
+      mbar_init(smem_u32(&ps->empty[s]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&ps->tfull[b]), 1);
+      mbar_init(smem_u32(&ps->tempty[b]), kEpiThreads / 32);
+      mbar_init(smem_u32(&ps->csfull[0][b]), 4);
+      mbar_init(smem_u32(&ps->csfull[1][b]), 4);
+    }
+    ps->abort = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmW);
+    tma_prefetch_desc(&tmX);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&ps->tmem_base), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ps->tmem_base;
+
+  if (warp < 4) {
+    setmaxnreg_dec<kProducerRegs>();
+    if (warp == 0 && lane == 0) {
+      // ------------------------------------------------ TMA producer
+      uint32_t it = 0;
+      for (int u = blockIdx.x; u < num_units && !*abort; u += gridDim.x) {
+        const int e = u / nbn, nb = u % nbn;
+        int r0, r1;
+        group_range(args, e, r0, r1);
+        for (int c0 = r0; c0 < r1 && !*abort; c0 += NT) {
+          const int cnt = min(NT, r1 - c0);
+          const int nbox = (cnt + 31) / 32;
+          for (int kb = 0; kb < nkb; ++kb, ++it) {
+            const int s = it % STAGES;
+            const uint32_t ph = (it / STAGES) & 1u;
+            if (!mbar_wait(smem_u32(&ps->empty[s]), ph ^ 1u, abort)) break;
+            const uint32_t w_addr = base + s * C::STAGE_BYTES;
+            const uint32_t bar = smem_u32(&ps->full[s]);
+            mbar_arrive_expect_tx(bar, C::W_BYTES + uint32_t(nbox) * 32u * kTileBytesPerRow);
+            tma_load_2d(w_addr, &tmW, bar, kb * kBK, e * args.N + nb * 128);
+            for (int i = 0; i < nbox; ++i)
+              tma_load_2d(w_addr + C::W_BYTES + i * 32 * kTileBytesPerRow, &tmX, bar, kb * kBK,
+                          c0 + 32 * i);
+          }
+        }
+      }
+    } else if (warp == 1 && lane == 0) {
+      // ------------------------------------------------ MMA issuer
+      uint32_t it = 0, kbc = 0;
+      for (int u = blockIdx.x; u < num_units && !*abort; u += gridDim.x) {
+        const int e = u / nbn;
+        int r0, r1;
+        group_range(args, e, r0, r1);
+        for (int c0 = r0; c0 < r1 && !*abort; c0 += NT) {
+          const int cnt = min(NT, r1 - c0);
+          const uint32_t n_mma = uint32_t((cnt + 15) / 16 * 16);
+          const uint32_t idesc = idesc_f8_e4m3_f32(128, n_mma);
+          for (int kb = 0; kb < nkb; ++kb, ++it, ++kbc) {
+            const int s = it % STAGES;
+            const uint32_t ph = (it / STAGES) & 1u;
+            const uint32_t b = kbc & 1u;
+            if (!mbar_wait(smem_u32(&ps->tempty[b]), ((kbc >> 1) & 1u) ^ 1u, abort)) break;
+            if (!mbar_wait(smem_u32(&ps->full[s]), ph, abort)) break;
+            tc_fence_after();
+            const uint32_t w_addr = base + s * C::STAGE_BYTES;
+            const uint32_t x_addr = w_addr + C::W_BYTES;
+            const uint32_t d = tmem + b * NT;
+#pragma unroll
+            for (int k = 0; k < kBK / 32; ++k)
+              mma_f8(d, sw128_kmajor_desc(w_addr + k * 32), sw128_kmajor_desc(x_addr + k * 32), idesc,
+                     k > 0 ? 1u : 0u);
+            mma_commit(smem_u32(&ps->empty[s]));
+            mma_commit(smem_u32(&ps->tfull[b]));
+          }
+        }
+      }
+    }
+  } else {
+    setmaxnreg_inc<kConsumerRegs>();
+    // ------------------------------------------------ promotion + epilogue
+    constexpr int CW = C::COLS_PER_WG;
+    const int ew = threadIdx.x - 128;    // 0..255
+    const int wg = ew >> 7;              // token-column half
+    const int t_in_wg = ew & 127;
+    const int quad = warp & 3;
+    const bool out32 = args.out_fp32 != 0;
+    float* cs = colscale + wg * CW;      // slot p of this warpgroup: cs[p * NT + j]
+    // Column scales move from the threads that load them to all threads of the
+    // warpgroup through a 2-slot ring guarded by mbarriers (4 warp arrivals per
+    // fill).  Slot kbc & 1 holds K-block kbc's scales; a thread only refills a slot
+    // after passing the wait for the other slot, which every thread arrives on only
+    // after it has finished reading this slot's previous contents.
+    uint32_t kbc = 0;
+    bool aborted = false;
+    for (int u = blockIdx.x; u < num_units && !aborted; u += gridDim.x) {
+      const int e = u / nbn, nb = u % nbn;
+      const int n = nb * 128 + quad * 32 + lane;        // weight row of this thread
+      const bool n_ok = n < args.N;
+      const float* sw_blk = args.sw + (int64_t(e) * nbn + nb) * nkb;
+      int r0, r1;
+      group_range(args, e, r0, r1);
+      for (int c0 = r0; c0 < r1; c0 += NT) {
+        const int cnt = min(NT, r1 - c0);
+        const int col0 = wg * CW;                       // first token column of this WG
+        // this thread loads the scale of token (c0 + col0 + t_in_wg), times sw[kb]
+        const bool tok_ok = (t_in_wg < CW) && (col0 + t_in_wg < cnt);
+        const float* sa_tok = args.sa + int64_t(tok_ok ? c0 + col0 + t_in_wg : 0) * nkb;
+        if (t_in_wg < CW) cs[(kbc & 1u) * NT + t_in_wg] = tok_ok ? __ldg(sa_tok) * __ldg(sw_blk) : 0.0f;
+        float next = (tok_ok && nkb > 1) ? __ldg(sa_tok + 1) * __ldg(sw_blk + 1) : 0.0f;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&ps->csfull[wg][kbc & 1u]));
+        float acc[CW];
+#pragma unroll
+        for (int j = 0; j < CW; ++j) acc[j] = 0.0f;
+        for (int kb = 0; kb < nkb; ++kb, ++kbc) {
+          const uint32_t b = kbc & 1u;
+          if (!mbar_wait(smem_u32(&ps->csfull[wg][b]), (kbc >> 1) & 1u, abort)) { aborted = true; break; }
+          if (!mbar_wait(smem_u32(&ps->tfull[b]), (kbc >> 1) & 1u, abort)) { aborted = true; break; }
+          tc_fence_after();
+          const float* csk = cs + b * NT;
+          const uint32_t taddr = tmem + (uint32_t(quad * 32) << 16) + b * NT + col0;
+#pragma unroll
+          for (int h = 0; h < CW / 32; ++h) {
+            uint32_t p[32];
+            tmem_ld32(taddr + h * 32, p);
+            tmem_ld_wait();
+            if (h == CW / 32 - 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(smem_u32(&ps->tempty[b]));
+            }
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+              const float4 sc = *reinterpret_cast<const float4*>(csk + h * 32 + j);
+              acc[h * 32 + j + 0] = fmaf(__uint_as_float(p[j + 0]), sc.x, acc[h * 32 + j + 0]);
+              acc[h * 32 + j + 1] = fmaf(__uint_as_float(p[j + 1]), sc.y, acc[h * 32 + j + 1]);
+              acc[h * 32 + j + 2] = fmaf(__uint_as_float(p[j + 2]), sc.z, acc[h * 32 + j + 2]);
+              acc[h * 32 + j + 3] = fmaf(__uint_as_float(p[j + 3]), sc.w, acc[h * 32 + j + 3]);
+            }
+          }
+          // fill the other slot with K-block kb+1's column scales
+          if (kb + 1 < nkb) {
+            if (t_in_wg < CW) cs[(b ^ 1u) * NT + t_in_wg] = next;
+            if (kb + 2 < nkb) next = tok_ok ? __ldg(sa_tok + kb + 2) * __ldg(sw_blk + kb + 2) : 0.0f;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&ps->csfull[wg][b ^ 1u]));
+          }
+        }
+        if (aborted) break;
+        if (n_ok) {
+          const int jmax = min(CW, cnt - col0);
+          const int64_t idx0 = int64_t(c0 + col0) * args.N + n;
+#pragma unroll
+          for (int j = 0; j < CW; ++j) {
+            if (j < jmax) {
+              const int64_t idx = idx0 + int64_t(j) * args.N;
+              if (out32)
+                reinterpret_cast<float*>(args.y)[idx] = acc[j];
+              else
+                reinterpret_cast<__nv_bfloat16*>(args.y)[idx] = __float2bfloat16_rn(acc[j]);
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (*abort) {
+    if (threadIdx.x == 0) settle_ns(200000);
+    __syncthreads();
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace fp8lin

@@ -1,0 +1,246 @@
+// quant.cuh -- memory-bound FP8 quantisers for sm_100a.
+//
+//  k_act_quant      per token, per 128-channel group ("FP8 推理提速 83.6%: DeepSeek-V3
+//                   在 AMD MI250 上的完整落地指南", 运行时: act_quant); one half-warp
+//                   owns one (row, group): 16 lanes x 16-byte loads = 128 bf16,
+//                   shuffle-xor amax over the 16 lanes, scale, cast, 8-byte stores.
+//  k_block_quant    one CTA per 128x128 weight block (same page, FP8 权重转换: e4m3
+//                   weights with a 128x128 block scale_inv).
+//  k_tensor_amax / k_tensor_cast / k_tensor_scale
+//                   per-tensor scaling ("ROCm 7 ... AITER", section 1.2: one scale per
+//                   tensor; "FP8 推理", Dynamic Scaling: scale = max|x| / 448): pass 1
+//                   folds the tensor's amax into the caller's scale slot with an
+//                   integer atomicMax, pass 2 casts (walking the tensor backwards so the
+//                   tail that pass 1 left in L2 is read from L2), pass 3 stores the scale.
+//
+// Arithmetic shared by all three (the pages' Q(x) with the scale as a divisor,
+// "量化：FP8 与混合精度推理", FP8 也需要 scale):
+//   s = max(fl32(amax / Fmax), 2^-126), or for ue8m0 the power of two 2^ceil(log2 .)
+//   q = cvt.rn.satfinite(fl32(x / s))  -- round to nearest even, clamp to +-Fmax.
+// For ue8m0 the division is a multiplication by the exact power of two 2^-e, which
+// rounds identically to the IEEE quotient (same exact value, one rounding).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace fp8lin {
+
+enum : int { kE4M3 = 0, kE5M2 = 1 };
+enum : int { kScaleFp32 = 0, kScaleUe8m0 = 1 };
+
+template <int FMT>
+struct FmtTraits;
+template <>
+struct FmtTraits<kE4M3> {
+  static constexpr float kMax = 448.0f;
+};
+template <>
+struct FmtTraits<kE5M2> {
+  static constexpr float kMax = 57344.0f;
+};
+
+// bf16 pair (little-endian: element 2i in the low half) -> two fp32, exactly.
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Scale and its exact reciprocal where one exists (ue8m0).  amax is finite, >= 0.
+template <int FMT, int SF>
+struct GroupScale {
+  float s;     // stored dequantisation multiplier
+  float rinv;  // 2^-e for ue8m0 (exact); unused for fp32 scales
+  __device__ __forceinline__ explicit GroupScale(float amax) {
+    const float v = __fdiv_rn(amax, FmtTraits<FMT>::kMax);
+    if (SF == kScaleFp32) {
+      s = fmaxf(v, 1.17549435082228750797e-38f);  // 2^-126
+      rinv = 0.0f;
+    } else {
+      // e = ceil(log2 v) from the bits of v; v == 0 or subnormal -> e <= -126 -> -126
+      const uint32_t b = __float_as_uint(v);
+      const int ex = int(b >> 23);
+      int e = (ex == 0) ? -126 : ex - 127 + ((b & 0x7FFFFFu) != 0u ? 1 : 0);
+      e = max(e, -126);
+      s = __uint_as_float(uint32_t(e + 127) << 23);
+      rinv = __uint_as_float(uint32_t(127 - e) << 23);
+    }
+  }
+  __device__ __forceinline__ float apply(float x) const {
+    if (SF == kScaleFp32) return __fdiv_rn(x, s);
+    return __fmul_rn(x, rinv);
+  }
+};
+
+// Two fp32 -> two FP8 codes in one 16-bit word; `lo` lands in the low byte.
+template <int FMT>
+__device__ __forceinline__ uint32_t cvt2(float lo, float hi) {
+  uint16_t r;
+  if (FMT == kE4M3)
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  else
+    asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// 8 bf16 (one uint4) -> 8 codes (one uint2) under scale sc.
+template <int FMT, int SF>
+__device__ __forceinline__ uint2 quant8(const uint4 v, const GroupScale<FMT, SF>& sc) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t c[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) c[i] = cvt2<FMT>(sc.apply(bf16_lo(w[i])), sc.apply(bf16_hi(w[i])));
+  return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+}
+
+__device__ __forceinline__ float amax8(const uint4 v, float a) {
+  a = fmaxf(a, fabsf(bf16_lo(v.x)));
+  a = fmaxf(a, fabsf(bf16_hi(v.x)));
+  a = fmaxf(a, fabsf(bf16_lo(v.y)));
+  a = fmaxf(a, fabsf(bf16_hi(v.y)));
+  a = fmaxf(a, fabsf(bf16_lo(v.z)));
+  a = fmaxf(a, fabsf(bf16_hi(v.z)));
+  a = fmaxf(a, fabsf(bf16_lo(v.w)));
+  a = fmaxf(a, fabsf(bf16_hi(v.w)));
+  return a;
+}
+
+__device__ __forceinline__ uint4 ldg_stream(const uint4* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+// ---------------------------------------------------------------- act_quant
+// Work item = (row m, group g) of 128 channels; a half-warp per item, each warp
+// iteration takes 2*UNROLL consecutive items (consecutive groups of a row are
+// contiguous in memory, so a warp reads 512 contiguous bytes per unrolled step).
+template <int FMT, int SF, int UNROLL>
+__global__ void __launch_bounds__(256) k_act_quant(const uint16_t* __restrict__ x, int64_t M,
+                                                   int64_t K, int64_t ldx, uint8_t* __restrict__ q,
+                                                   float* __restrict__ s) {
+  const int64_t ng = (K + 127) / 128;
+  const int64_t total = M * ng;
+  const int lane = threadIdx.x & 31;
+  const int half = lane >> 4, hl = lane & 15;
+  const int64_t warp = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarp = (int64_t(gridDim.x) * blockDim.x) >> 5;
+
+  for (int64_t base = warp * (2 * UNROLL); base < total; base += nwarp * (2 * UNROLL)) {
+    uint4 v[UNROLL];
+    int64_t row[UNROLL], col[UNROLL];
+    bool ok[UNROLL];
+    // one division per warp step; the 2*UNROLL items that follow are stepped to
+    const int64_t m0 = base / ng;
+    const int64_t g0 = base - m0 * ng;
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+      const int64_t item = base + 2 * u + half;
+      int64_t m = m0, g = g0 + 2 * u + half;
+      while (g >= ng) { g -= ng; ++m; }   // at most 2*UNROLL steps
+      row[u] = m;
+      col[u] = g * 128 + hl * 8;
+      ok[u] = (item < total) && (col[u] < K);
+      v[u] = ok[u] ? ldg_stream(reinterpret_cast<const uint4*>(x + m * ldx + col[u]))
+                   : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+      float a = amax8(v[u], 0.0f);
+      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 8));
+      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 4));
+      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+      const GroupScale<FMT, SF> sc(a);
+      if (ok[u]) {
+        *reinterpret_cast<uint2*>(q + row[u] * K + col[u]) = quant8<FMT, SF>(v[u], sc);
+        if (hl == 0) s[row[u] * ng + (col[u] >> 7)] = sc.s;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------- 128x128 block quant
+// One CTA (256 threads) per block: thread t covers columns (t & 15) * 8 .. +8 of
+// rows (t >> 4) + 16 i, i = 0..7, so each warp reads two full 256-byte row
+// segments per load instruction.
+template <int FMT, int SF>
+__global__ void __launch_bounds__(256) k_block_quant(const uint16_t* __restrict__ w, int64_t N,
+                                                     int64_t K, uint8_t* __restrict__ q,
+                                                     float* __restrict__ s_inv) {
+  __shared__ float red[8];
+  const int64_t nbk = (K + 127) / 128;
+  const int64_t bn = blockIdx.y, bk = blockIdx.x;
+  const int t = threadIdx.x;
+  const int64_t c = bk * 128 + (t & 15) * 8;
+  const bool col_ok = c < K;
+  uint4 v[8];
+  float a = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int64_t r = bn * 128 + (t >> 4) + 16 * i;
+    const bool ok = col_ok && r < N;
+    v[i] = ok ? ldg_stream(reinterpret_cast<const uint4*>(w + r * K + c)) : make_uint4(0u, 0u, 0u, 0u);
+    a = amax8(v[i], a);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+  if ((t & 31) == 0) red[t >> 5] = a;
+  __syncthreads();
+  a = red[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) a = fmaxf(a, red[i]);
+  const GroupScale<FMT, SF> sc(a);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int64_t r = bn * 128 + (t >> 4) + 16 * i;
+    if (col_ok && r < N) *reinterpret_cast<uint2*>(q + r * K + c) = quant8<FMT, SF>(v[i], sc);
+  }
+  if (t == 0) s_inv[bn * nbk + bk] = sc.s;
+}
+
+// ------------------------------------------------------------ per-tensor
+// Pass 1: amax of n8*8 elements folded into *amax_bits (non-negative floats order
+// like their bit patterns, so an unsigned atomicMax is an exact float max).
+__global__ void __launch_bounds__(256) k_tensor_amax(const uint16_t* __restrict__ x, int64_t n8,
+                                                     unsigned int* amax_bits) {
+  __shared__ float red[8];
+  float a = 0.0f;
+  const uint4* p = reinterpret_cast<const uint4*>(x);
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+       i += int64_t(gridDim.x) * blockDim.x)
+    a = amax8(ldg_stream(p + i), a);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int i = 1; i < 8; ++i) a = fmaxf(a, red[i]);
+    atomicMax(amax_bits, __float_as_uint(a));
+  }
+}
+
+// Pass 2: cast with the scale derived from the finished amax; indices run from the
+// end of the tensor backwards.
+template <int FMT, int SF>
+__global__ void __launch_bounds__(256) k_tensor_cast(const uint16_t* __restrict__ x, int64_t n8,
+                                                     const unsigned int* amax_bits,
+                                                     uint8_t* __restrict__ q) {
+  const GroupScale<FMT, SF> sc(__uint_as_float(*amax_bits));
+  const uint4* p = reinterpret_cast<const uint4*>(x);
+  uint2* o = reinterpret_cast<uint2*>(q);
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+       i += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t j = n8 - 1 - i;
+    o[j] = quant8<FMT, SF>(ldg_stream(p + j), sc);
+  }
+}
+
+// Pass 3: replace the amax bits with the scale.
+template <int FMT, int SF>
+__global__ void k_tensor_scale(unsigned int* slot) {
+  const GroupScale<FMT, SF> sc(__uint_as_float(*slot));
+  *reinterpret_cast<float*>(slot) = sc.s;
+}
+
+}  // namespace fp8lin

@@ -1,0 +1,147 @@
+/*
+ * fp8lin.h -- C ABI of the B200 (sm_100a) FP8 W8A8 linear-layer library.
+ *
+ * The library implements the linear layer that the DeepSeek-V3 deployment page
+ * ("FP8 推理提速 83.6%: DeepSeek-V3 在 AMD MI250 上的完整落地指南", section 运行时)
+ * runs when dtype is fp8:
+ *     x, scale = act_quant(x, block_size, scale_fmt)   # per token, per 128 channels
+ *     y        = fp8_gemm(x, scale, weight, weight.scale)
+ * with weights stored as E4M3 codes plus one fp32 scale_inv per 128x128 block
+ * (same page, FP8 权重转换命令与关键配置参数), and the MoE variant over 256 routed
+ * experts with 8 active per token (same page, 官方配置中最关键的四个参数).
+ *
+ * Conventions shared by every entry point
+ *  - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *    allocates and frees no device memory and keeps no per-call state.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Every call only enqueues work on that stream and returns; results are ready
+ *    when the stream reaches that point.
+ *  - Arguments are validated on the host before anything is launched; a rejected
+ *    call returns a non-zero fp8_status and enqueues nothing.  A failed launch
+ *    returns FP8_ERR_CUDA.  Nothing aborts or throws across the ABI.
+ *  - Row-major layouts throughout.  "codes" are one byte per element (E4M3 or
+ *    E5M2 bit patterns).  Scales are fp32 dequantisation multipliers:
+ *    x ~= decode(code) * s  ("量化：FP8 与混合精度推理", FP8 也需要 scale).
+ *  - Rounding: q = saturate(round_to_nearest_even(fl32(x / s))) to +-Fmax, so no
+ *    code is ever Inf (E4M3 Fmax = 448, E5M2 Fmax = 57344; "LLM 推理的 FP8 混合精度
+ *    工程 2026", section 2).  s = max(fl32(amax / Fmax), 2^-126); with
+ *    FP8_SCALE_UE8M0 s is that value rounded up to a power of two (stored as fp32).
+ *  - Pipelined waits inside the GEMM kernels are bounded (about 2 s); a wait that
+ *    runs out sets a device-side error word that fp8_device_error() reports.
+ */
+#ifndef FP8LIN_H
+#define FP8LIN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FP8_OK = 0,
+    FP8_ERR_INVALID_ARG = 1,   /* null pointer, bad enum value, negative size */
+    FP8_ERR_SHAPE = 2,         /* shape outside what the operation supports      */
+    FP8_ERR_ALIGNMENT = 3,     /* pointer or leading dimension misaligned        */
+    FP8_ERR_UNSUPPORTED = 4,   /* valid request this build does not implement    */
+    FP8_ERR_CUDA = 5,          /* a CUDA runtime call or launch failed           */
+    FP8_ERR_TIMEOUT = 6        /* a bounded device-side wait ran out             */
+} fp8_status;
+
+typedef enum { FP8_E4M3 = 0, FP8_E5M2 = 1 } fp8_format;
+typedef enum { FP8_SCALE_FP32 = 0, FP8_SCALE_UE8M0 = 1 } fp8_scale_fmt;
+typedef enum { FP8_OUT_BF16 = 0, FP8_OUT_FP32 = 1 } fp8_out_dtype;
+
+/*
+ * fp8_act_quant -- dynamic per-token, per-group activation quantisation
+ * (DeepSeek-V3 page, 运行时: act_quant per token per 128 channels; "FP8 推理",
+ * Dynamic Scaling: scale = max|x| / 448 from the current batch).
+ *
+ *   x      bf16 [M][ldx] (only the first K columns are read); 16-byte aligned.
+ *   M, K   rows and columns, M >= 0, K > 0, K % 16 == 0.  The last group of a row
+ *          may be shorter than `group` (its amax covers the valid columns only).
+ *   ldx    row stride of x in elements, ldx >= K, ldx % 8 == 0.
+ *   group  channels per scale; 128 is the supported value.
+ *   fmt    FP8_E4M3 or FP8_E5M2 codes.
+ *   scale_fmt  FP8_SCALE_FP32 or FP8_SCALE_UE8M0.
+ *   q      codes [M][K] (dense, row stride K); 16-byte aligned.
+ *   s      fp32 scales [M][ceil(K/group)] (dense).
+ * Returns FP8_OK, or INVALID_ARG / SHAPE / ALIGNMENT / UNSUPPORTED / CUDA.
+ * M == 0 is a no-op.
+ */
+int fp8_act_quant(const void* x, int64_t M, int64_t K, int64_t ldx, int group,
+                  int fmt, int scale_fmt, void* q, float* s, void* stream);
+
+/*
+ * fp8_weight_quant -- weight quantisation with one scale_inv per block x block
+ * tile (DeepSeek-V3 page, FP8 权重转换命令与关键配置参数: e4m3 weights, 128x128
+ * block scales), or with one scale for the whole tensor when block == 0 (the
+ * per-tensor OCP scaling the ROCm page contrasts with block scaling, section 1.2;
+ * E5M2 allowed here, Fmax 57344).
+ *
+ *   w      bf16 [N][K] (dense); 16-byte aligned.
+ *   N, K   N >= 0, K > 0, K % 16 == 0.  Edge blocks may be partial.
+ *   block  128, or 0 for per-tensor.
+ *   q      codes [N][K]; 16-byte aligned.
+ *   s_inv  fp32 [ceil(N/128)][ceil(K/128)] for block == 128, fp32 [1] for block == 0.
+ *          In per-tensor mode s_inv[0] also serves, in stream order, as the amax
+ *          accumulator of the first pass, so it must not alias w or q.
+ * Returns FP8_OK or an error status; N == 0 is a no-op.
+ */
+int fp8_weight_quant(const void* w, int64_t N, int64_t K, int block, int fmt,
+                     int scale_fmt, void* q, float* s_inv, void* stream);
+
+/*
+ * fp8_block_gemm -- block-scaled FP8 GEMM with fp32 accumulation
+ * (DeepSeek-V3 page, 运行时: fp8_gemm(x, scale, weight, weight.scale);
+ * "LLM 推理的 FP8 混合精度工程 2026", section 3: FP32 accumulation):
+ *
+ *   y[m][n] = sum_{kb < K/128} sa[m][kb] * sw[n/128][kb] *
+ *             sum_{k in block kb} dec(qa[m][k]) * dec(qw[n][k])
+ *
+ *   qa     E4M3 codes [M][K]; 16-byte aligned.
+ *   sa     fp32 [M][K/128] (act_quant's layout).
+ *   qw     E4M3 codes [N][K]; 16-byte aligned.
+ *   sw     fp32 [ceil(N/128)][K/128] (weight_quant's layout).
+ *   M >= 0, N > 0 with N % 16 == 0, K > 0 with K % 128 == 0.
+ *   out_dtype  FP8_OUT_BF16 (round to nearest even) or FP8_OUT_FP32.
+ *   y      [M][N] of out_dtype; 16-byte aligned.
+ * Each 128-deep K-block is one tensor-core partial product that is scaled and
+ * added into an fp32 accumulator (per-K-block promotion).
+ */
+int fp8_block_gemm(const void* qa, const float* sa, const void* qw, const float* sw,
+                   int64_t M, int64_t N, int64_t K, int out_dtype, void* y, void* stream);
+
+/*
+ * fp8_grouped_gemm -- the same GEMM per MoE expert over expert-sorted rows
+ * (ROCm page, section 2.3: block-scale fused MoE; DeepSeek-V3 page: 256 routed
+ * experts, 8 active per token).  Row m of qa belongs to expert e when
+ * group_offsets[e] <= m < group_offsets[e+1]; it is multiplied by qw[e].
+ *
+ *   qa     E4M3 codes [total_M][K]; sa fp32 [total_M][K/128].
+ *   qw     E4M3 codes [E][N][K]; sw fp32 [E][ceil(N/128)][K/128].
+ *   group_offsets  DEVICE int32 [E+1], non-decreasing, [0] == 0,
+ *          [E] <= total_M.  Not read on the host (no synchronisation).
+ *   E > 0, total_M >= 0, N % 16 == 0, K % 128 == 0.
+ *   y      [total_M][N] of out_dtype.  Rows outside every group are not written.
+ */
+int fp8_grouped_gemm(const void* qa, const float* sa, const void* qw, const float* sw,
+                     const int32_t* group_offsets, int64_t E, int64_t total_M,
+                     int64_t N, int64_t K, int out_dtype, void* y, void* stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* fp8_status_string(int status);
+
+/*
+ * fp8_device_error -- synchronises `stream`, then reads and clears the
+ * library's device-side error word on the current device.  Returns FP8_OK, or
+ * FP8_ERR_TIMEOUT if a bounded wait in an earlier kernel ran out (that kernel
+ * skipped its remaining work and returned), or FP8_ERR_CUDA.
+ */
+int fp8_device_error(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8LIN_H */

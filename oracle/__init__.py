@@ -46,6 +46,8 @@ def lib():
         L.orc_act_quant.argtypes = [vp, i64, i64, i64, i64, ctypes.c_int, ctypes.c_int, vp, vp]
         L.orc_weight_quant_block.restype = None
         L.orc_weight_quant_block.argtypes = [vp, i64, i64, i64, ctypes.c_int, ctypes.c_int, vp, vp]
+        L.orc_cast_with_scale.restype = None
+        L.orc_cast_with_scale.argtypes = [vp, i64, ctypes.c_float, ctypes.c_int, vp]
         L.orc_tensor_quant.restype = None
         L.orc_tensor_quant.argtypes = [vp, i64, ctypes.c_int, ctypes.c_int, vp, vp]
         L.orc_gemm_rows.restype = None
@@ -135,6 +137,14 @@ def tensor_quant(x, fmt: int = E4M3, scale_fmt: int = SCALE_FP32):
     s = np.empty((1,), dtype=np.float32)
     lib().orc_tensor_quant(_ptr(xb), xb.size, fmt, scale_fmt, _ptr(q), _ptr(s))
     return q, s
+
+
+def cast_with_scale(x, s: float, fmt: int = E4M3):
+    """Codes of bf16 x under a given scale: FP8Cast(x / s), same shape as x."""
+    xb = _bf16_bits(x)
+    q = np.empty(xb.shape, dtype=np.uint8)
+    lib().orc_cast_with_scale(_ptr(xb), xb.size, float(s), fmt, _ptr(q))
+    return q
 
 
 # ------------------------------------------------------------------ GEMM

@@ -205,6 +205,13 @@ void orc_weight_quant_block(const uint16_t *w, int64_t N, int64_t K, int64_t blo
     }
 }
 
+/* The cast step under a given scale: q[i] = FP8Cast(x[i] / s) ([P5] FP8 也需要
+ * scale), one IEEE fp32 division then the encoder above. */
+void orc_cast_with_scale(const uint16_t *x, int64_t n, float s, int fmt, uint8_t *q)
+{
+    for (int64_t i = 0; i < n; ++i) q[i] = orc_encode(bf16_to_f32(x[i]) / s, fmt);
+}
+
 /* Per-tensor quantisation ([P1] 1.2 OCP-FP8 one scale per tensor; [P3] scale =
  * max(|tensor|)/448; [P2] Fmax 57344 for E5M2).  One scale for all n elements. */
 void orc_tensor_quant(const uint16_t *x, int64_t n, int fmt, int scale_fmt,
@@ -214,7 +221,7 @@ void orc_tensor_quant(const uint16_t *x, int64_t n, int fmt, int scale_fmt,
     for (int64_t i = 0; i < n; ++i) amax = amax_accum(amax, bf16_to_f32(x[i]));
     float sc = orc_scale_from_amax(amax, fmt, scale_fmt);
     s[0] = sc;
-    for (int64_t i = 0; i < n; ++i) q[i] = orc_encode(bf16_to_f32(x[i]) / sc, fmt);
+    orc_cast_with_scale(x, n, sc, fmt, q);
 }
 
 /* -------------------------------------------------------------------- GEMM */

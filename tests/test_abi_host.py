@@ -1,0 +1,93 @@
+"""Host-only checks of the C ABI: the library loads, exports every function the
+header declares, and rejects bad arguments with the documented status before
+touching the GPU (every call below fails validation, so nothing is launched)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import fp8_block_scaled_12_b200 as F
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fp8lin.h")
+
+OK, INVALID, SHAPE, ALIGN, UNSUP, CUDA, TIMEOUT = range(7)
+FAKE = 0x7F0000000000       # 16-byte aligned, never dereferenced
+S = None                    # default stream
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fp8_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_four_operations():
+    names = declared_functions()
+    for n in ("fp8_act_quant", "fp8_weight_quant", "fp8_block_gemm", "fp8_grouped_gemm"):
+        assert n in names
+
+
+def test_library_exports_every_declared_function():
+    lib = ctypes.CDLL(F.LIB_PATH)
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+
+
+def test_status_strings():
+    assert F.fp8_status_string(OK) == "ok"
+    for c in range(1, 7):
+        assert F.fp8_status_string(c) not in ("ok", "unknown status")
+    assert F.fp8_status_string(99) == "unknown status"
+
+
+def aq(*a):
+    return F.lib.fp8_act_quant(*a)
+
+
+def test_act_quant_validation():
+    # (x, M, K, ldx, group, fmt, sf, q, s, stream)
+    assert aq(FAKE, -1, 128, 128, 128, 0, 0, FAKE, FAKE, S) == INVALID
+    assert aq(FAKE, 4, 128, 64, 128, 0, 0, FAKE, FAKE, S) == INVALID        # ldx < K
+    assert aq(FAKE, 4, 128, 128, 128, 2, 0, FAKE, FAKE, S) == INVALID       # bad format
+    assert aq(FAKE, 4, 128, 128, 128, 0, 7, FAKE, FAKE, S) == INVALID       # bad scale format
+    assert aq(FAKE, 4, 128, 128, 32, 0, 0, FAKE, FAKE, S) == UNSUP          # group 32 not built
+    assert aq(FAKE, 4, 136, 136, 128, 0, 0, FAKE, FAKE, S) == SHAPE         # K % 16
+    assert aq(None, 4, 128, 128, 128, 0, 0, FAKE, FAKE, S) == INVALID       # null x
+    assert aq(FAKE + 8, 4, 128, 128, 128, 0, 0, FAKE, FAKE, S) == ALIGN     # x not 16-byte aligned
+    assert aq(FAKE, 4, 128, 132, 128, 0, 0, FAKE, FAKE, S) == ALIGN         # ldx % 8
+    assert aq(FAKE, 0, 128, 128, 128, 0, 0, None, None, S) == OK            # M == 0: no-op
+
+
+def test_weight_quant_validation():
+    wq = F.lib.fp8_weight_quant
+    assert wq(FAKE, 256, 256, 64, 0, 0, FAKE, FAKE, S) == UNSUP             # block 64 not built
+    assert wq(FAKE, 256, 250, 128, 0, 0, FAKE, FAKE, S) == SHAPE
+    assert wq(FAKE, 256, 256, 128, 0, 0, FAKE, None, S) == INVALID
+    assert wq(FAKE, 256, 256, 128, 0, 0, FAKE + 4, FAKE, S) == ALIGN
+    assert wq(FAKE, 0, 256, 0, 1, 0, None, None, S) == OK
+
+
+def test_gemm_validation():
+    g = F.lib.fp8_block_gemm
+    # (qa, sa, qw, sw, M, N, K, out, y, stream)
+    assert g(FAKE, FAKE, FAKE, FAKE, 16, 256, 200, 0, FAKE, S) == SHAPE     # K % 128
+    assert g(FAKE, FAKE, FAKE, FAKE, 16, 100, 256, 0, FAKE, S) == SHAPE     # N % 16
+    assert g(FAKE, FAKE, FAKE, FAKE, 16, 256, 256, 5, FAKE, S) == INVALID   # out dtype
+    assert g(None, FAKE, FAKE, FAKE, 16, 256, 256, 0, FAKE, S) == INVALID
+    assert g(FAKE, FAKE, FAKE + 1, FAKE, 16, 256, 256, 0, FAKE, S) == ALIGN
+    assert g(FAKE, FAKE, FAKE, FAKE, 0, 256, 256, 0, None, S) == OK         # M == 0
+    gg = F.lib.fp8_grouped_gemm
+    # (qa, sa, qw, sw, off, E, total_M, N, K, out, y, stream)
+    assert gg(FAKE, FAKE, FAKE, FAKE, None, 4, 16, 256, 256, 0, FAKE, S) == INVALID
+    assert gg(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 16, 256, 256, 0, FAKE, S) == INVALID
+    assert gg(FAKE, FAKE, FAKE, FAKE, FAKE + 2, 4, 16, 256, 256, 0, FAKE, S) == ALIGN
+    assert gg(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 0, 256, 256, 0, None, S) == OK
+
+
+def test_python_binding_rejects_host_tensors():
+    import torch
+    x = torch.zeros(4, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        F.fp8_act_quant(x, torch.zeros(4, 128, dtype=torch.uint8), torch.zeros(4, 1))
