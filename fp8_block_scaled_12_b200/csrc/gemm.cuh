@@ -46,7 +46,7 @@ constexpr uint32_t kTileBytesPerRow = 128;
 // (launch bounds 384 x 1); the split must not exceed that pool:
 // 128 * kProducerRegs + 256 * kConsumerRegs == 384 * kLaunchRegs.
 constexpr uint32_t kLaunchRegs = 168;
-constexpr uint32_t kProducerRegs = 56;
+constexpr uint32_t kProducerRegs = 48;
 constexpr uint32_t kConsumerRegs = 224;
 static_assert(128 * kProducerRegs + 256 * kConsumerRegs <= 384 * kLaunchRegs, "register split exceeds pool");
 
@@ -208,9 +208,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool cols_any = n0 < args.N;
       const float* sa_row = args.sa + (row_ok ? m : 0) * nkb;
       const float* sw_blk = args.sw + int64_t(cols_any ? n0 / 128 : 0) * nkb;
-      float acc[128];
+      uint64_t acc[64];                  // 128 fp32 accumulators as packed pairs
 #pragma unroll
-      for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
+      for (int j = 0; j < 64; ++j) acc[j] = 0ull;
       float sa_next = row_ok ? __ldg(sa_row) : 0.0f;
       float sw_next = cols_any ? __ldg(sw_blk) : 0.0f;
       bool aborted = false;
@@ -235,10 +235,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&ps->tempty[b]));
           }
+          const uint64_t s2 = pack2(scale, scale);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            acc[h * 64 + j] = fmaf(__uint_as_float(p0[j]), scale, acc[h * 64 + j]);
-            acc[h * 64 + 32 + j] = fmaf(__uint_as_float(p1[j]), scale, acc[h * 64 + 32 + j]);
+          for (int j = 0; j < 16; ++j) {
+            ffma2(acc[h * 32 + j], p0[2 * j], p0[2 * j + 1], s2);
+            ffma2(acc[h * 32 + 16 + j], p1[2 * j], p1[2 * j + 1], s2);
           }
         }
       }
@@ -246,7 +247,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (row_ok && cols_any) {
 #pragma unroll
         for (int j = 0; j < 128; j += 8) {
-          if (n0 + j < args.N) store8(args.y, out32, m * args.N + n0 + j, &acc[j]);
+          float v[8];
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const float2 f = unpack2(acc[j / 2 + t]);
+            v[2 * t] = f.x;
+            v[2 * t + 1] = f.y;
+          }
+          if (n0 + j < args.N) store8(args.y, out32, m * args.N + n0 + j, v);
         }
       }
     }
@@ -427,9 +435,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         float next = (tok_ok && nkb > 1) ? __ldg(sa_tok + 1) * __ldg(sw_blk + 1) : 0.0f;
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&ps->csfull[wg][kbc & 1u]));
-        float acc[CW];
+        uint64_t acc[CW / 2];              // CW fp32 accumulators as packed pairs
 #pragma unroll
-        for (int j = 0; j < CW; ++j) acc[j] = 0.0f;
+        for (int j = 0; j < CW / 2; ++j) acc[j] = 0ull;
         for (int kb = 0; kb < nkb; ++kb, ++kbc) {
           const uint32_t b = kbc & 1u;
           if (!mbar_wait(smem_u32(&ps->csfull[wg][b]), (kbc >> 1) & 1u, abort)) { aborted = true; break; }
@@ -449,11 +457,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
 #pragma unroll
             for (int j = 0; j < 32; j += 4) {
-              const float4 sc = *reinterpret_cast<const float4*>(csk + h * 32 + j);
-              acc[h * 32 + j + 0] = fmaf(__uint_as_float(p[j + 0]), sc.x, acc[h * 32 + j + 0]);
-              acc[h * 32 + j + 1] = fmaf(__uint_as_float(p[j + 1]), sc.y, acc[h * 32 + j + 1]);
-              acc[h * 32 + j + 2] = fmaf(__uint_as_float(p[j + 2]), sc.z, acc[h * 32 + j + 2]);
-              acc[h * 32 + j + 3] = fmaf(__uint_as_float(p[j + 3]), sc.w, acc[h * 32 + j + 3]);
+              const ulonglong2 sc = *reinterpret_cast<const ulonglong2*>(csk + h * 32 + j);
+              ffma2(acc[(h * 32 + j) / 2], p[j], p[j + 1], sc.x);
+              ffma2(acc[(h * 32 + j) / 2 + 1], p[j + 2], p[j + 3], sc.y);
             }
           }
           // fill the other slot with K-block kb+1's column scales
@@ -472,10 +478,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < CW; ++j) {
             if (j < jmax) {
               const int64_t idx = idx0 + int64_t(j) * args.N;
+              const float2 f = unpack2(acc[j / 2]);
+              const float v = (j & 1) ? f.y : f.x;
               if (out32)
-                reinterpret_cast<float*>(args.y)[idx] = acc[j];
+                reinterpret_cast<float*>(args.y)[idx] = v;
               else
-                reinterpret_cast<__nv_bfloat16*>(args.y)[idx] = __float2bfloat16_rn(acc[j]);
+                reinterpret_cast<__nv_bfloat16*>(args.y)[idx] = __float2bfloat16_rn(v);
             }
           }
         }
