@@ -120,10 +120,10 @@ int launch_wide(const void* qa, const void* qw, const GemmArgs& a, cudaStream_t 
 template <int FMT, int SF>
 int launch_act_quant(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q, float* s,
                      cudaStream_t st) {
-  constexpr int U = 4;
+  constexpr int U = 2;
   const int64_t ng = (K + 127) / 128;
   const int64_t items = M * ng;
-  const int64_t per_block = (256 / 32) * 2 * U;
+  const int64_t per_block = (256 / 32) * 8 * U;
   int64_t blocks = (items + per_block - 1) / per_block;
   const int64_t cap = int64_t(num_sms()) * 8;
   if (blocks > cap) blocks = cap;

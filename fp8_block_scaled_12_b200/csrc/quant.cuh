@@ -1,9 +1,9 @@
 // quant.cuh -- memory-bound FP8 quantisers for sm_100a.
 //
 //  k_act_quant      per token, per 128-channel group ("FP8 推理提速 83.6%: DeepSeek-V3
-//                   在 AMD MI250 上的完整落地指南", 运行时: act_quant); one half-warp
-//                   owns one (row, group): 16 lanes x 16-byte loads = 128 bf16,
-//                   shuffle-xor amax over the 16 lanes, scale, cast, 8-byte stores.
+//                   在 AMD MI250 上的完整落地指南", 运行时: act_quant); four lanes own
+//                   one (row, group): 4 x 16-byte loads each, two shuffle-xor steps for
+//                   the amax, scale, cast, 16-byte stores.
 //  k_block_quant    one CTA per 128x128 weight block (same page, FP8 权重转换: e4m3
 //                   weights with a 128x128 block scale_inv).
 //  k_tensor_amax / k_tensor_cast / k_tensor_scale
@@ -17,8 +17,7 @@
 // "量化：FP8 与混合精度推理", FP8 也需要 scale):
 //   s = max(fl32(amax / Fmax), 2^-126), or for ue8m0 the power of two 2^ceil(log2 .)
 //   q = cvt.rn.satfinite(fl32(x / s))  -- round to nearest even, clamp to +-Fmax.
-// For ue8m0 the division is a multiplication by the exact power of two 2^-e, which
-// rounds identically to the IEEE quotient (same exact value, one rounding).
+// (GroupScale below says how the division is carried out.)
 #pragma once
 
 #include <cstdint>
@@ -44,16 +43,33 @@ struct FmtTraits<kE5M2> {
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// Scale and its exact reciprocal where one exists (ue8m0).  amax is finite, >= 0.
+// Scale of a group and what the cast needs to divide by it.  amax is finite, >= 0.
+//
+// fp32 scales: x / s by a correctly rounded reciprocal r = 1/s' and one residual
+// correction (Markstein's division: q0 = x' r, e = x' - q0 s' exactly by FMA,
+// q = q0 + e r, then the sign of x), 4 FP operations and a sign merge instead of an
+// IEEE division per element.  Groups
+// with s < 2^-64 first scale x and s by 2^64 (exact) so every residual that can
+// decide a code stays a normal number.  For every bf16 amax and every bf16 x with
+// |x| <= amax this gives the same FP8 code as fl32(x / s) rounded to nearest even
+// (checked exhaustively, E4M3 and E5M2: tests/test_division_identity.py); the fp32
+// quotients themselves may differ only where they are far below the smallest FP8
+// subnormal.
+// ue8m0 scales: a multiplication by the exact power of two 2^-e, which rounds
+// identically to the IEEE quotient (same exact value, one rounding).
 template <int FMT, int SF>
 struct GroupScale {
   float s;     // stored dequantisation multiplier
-  float rinv;  // 2^-e for ue8m0 (exact); unused for fp32 scales
+  float rinv;  // fp32: RN(1 / (s * pre)); ue8m0: 2^-e (exact)
+  float pre;   // fp32: 1 or 2^64; ue8m0: unused
+  float ss;    // fp32: s * pre (exact)
   __device__ __forceinline__ explicit GroupScale(float amax) {
     const float v = __fdiv_rn(amax, FmtTraits<FMT>::kMax);
     if (SF == kScaleFp32) {
       s = fmaxf(v, 1.17549435082228750797e-38f);  // 2^-126
-      rinv = 0.0f;
+      pre = (s < 5.42101086242752217004e-20f) ? 18446744073709551616.0f : 1.0f;   // 2^-64 : 2^64
+      ss = __fmul_rn(s, pre);
+      rinv = __frcp_rn(ss);
     } else {
       // e = ceil(log2 v) from the bits of v; v == 0 or subnormal -> e <= -126 -> -126
       const uint32_t b = __float_as_uint(v);
@@ -62,10 +78,19 @@ struct GroupScale {
       e = max(e, -126);
       s = __uint_as_float(uint32_t(e + 127) << 23);
       rinv = __uint_as_float(uint32_t(127 - e) << 23);
+      pre = 1.0f;
+      ss = s;
     }
   }
   __device__ __forceinline__ float apply(float x) const {
-    if (SF == kScaleFp32) return __fdiv_rn(x, s);
+    if (SF == kScaleFp32) {
+      const float xs = __fmul_rn(x, pre);
+      const float q0 = __fmul_rn(xs, rinv);
+      const float e = __fmaf_rn(-q0, ss, xs);
+      // the sign of the quotient is the sign of x (s > 0); the correction step would
+      // turn a -0 quotient into +0
+      return copysignf(__fmaf_rn(e, rinv, q0), x);
+    }
     return __fmul_rn(x, rinv);
   }
 };
@@ -112,9 +137,11 @@ __device__ __forceinline__ uint4 ldg_stream(const uint4* p) {
 }
 
 // ---------------------------------------------------------------- act_quant
-// Work item = (row m, group g) of 128 channels; a half-warp per item, each warp
-// iteration takes 2*UNROLL consecutive items (consecutive groups of a row are
-// contiguous in memory, so a warp reads 512 contiguous bytes per unrolled step).
+// Work item = (row m, group g) of 128 channels, owned by 4 consecutive lanes: lane
+// quarter t holds channels [32t, 32t+32) of the group (four 16-byte loads), so the
+// group amax needs two shuffles and each lane casts 32 values with one scale.  A
+// warp takes 8 consecutive items per step (consecutive groups of a row are adjacent
+// in memory: a 2 KB contiguous span), and UNROLL steps per loop iteration.
 template <int FMT, int SF, int UNROLL>
 __global__ void __launch_bounds__(256) k_act_quant(const uint16_t* __restrict__ x, int64_t M,
                                                    int64_t K, int64_t ldx, uint8_t* __restrict__ q,
@@ -122,39 +149,51 @@ __global__ void __launch_bounds__(256) k_act_quant(const uint16_t* __restrict__ 
   const int64_t ng = (K + 127) / 128;
   const int64_t total = M * ng;
   const int lane = threadIdx.x & 31;
-  const int half = lane >> 4, hl = lane & 15;
+  const int slot = lane >> 2, qt = lane & 3;
   const int64_t warp = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarp = (int64_t(gridDim.x) * blockDim.x) >> 5;
 
-  for (int64_t base = warp * (2 * UNROLL); base < total; base += nwarp * (2 * UNROLL)) {
-    uint4 v[UNROLL];
+  for (int64_t base = warp * (8 * UNROLL); base < total; base += nwarp * (8 * UNROLL)) {
+    uint4 v[UNROLL][4];
     int64_t row[UNROLL], col[UNROLL];
-    bool ok[UNROLL];
-    // one division per warp step; the 2*UNROLL items that follow are stepped to
+    bool item_ok[UNROLL];
+    // one division per warp step; the items that follow are stepped to
     const int64_t m0 = base / ng;
     const int64_t g0 = base - m0 * ng;
 #pragma unroll
     for (int u = 0; u < UNROLL; ++u) {
-      const int64_t item = base + 2 * u + half;
-      int64_t m = m0, g = g0 + 2 * u + half;
-      while (g >= ng) { g -= ng; ++m; }   // at most 2*UNROLL steps
+      const int64_t item = base + 8 * u + slot;
+      int64_t m = m0, g = g0 + 8 * u + slot;
+      while (g >= ng) { g -= ng; ++m; }   // at most 8*UNROLL steps
       row[u] = m;
-      col[u] = g * 128 + hl * 8;
-      ok[u] = (item < total) && (col[u] < K);
-      v[u] = ok[u] ? ldg_stream(reinterpret_cast<const uint4*>(x + m * ldx + col[u]))
-                   : make_uint4(0u, 0u, 0u, 0u);
+      col[u] = g * 128 + qt * 32;
+      item_ok[u] = item < total;
+      const uint16_t* src = x + m * ldx + col[u];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const bool ok = item_ok[u] && (col[u] + 8 * j < K);
+        v[u][j] = ok ? __ldg(reinterpret_cast<const uint4*>(src + 8 * j)) : make_uint4(0u, 0u, 0u, 0u);
+      }
     }
 #pragma unroll
     for (int u = 0; u < UNROLL; ++u) {
-      float a = amax8(v[u], 0.0f);
-      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 8));
-      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 4));
-      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+      float a = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) a = amax8(v[u][j], a);
       a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
       const GroupScale<FMT, SF> sc(a);
-      if (ok[u]) {
-        *reinterpret_cast<uint2*>(q + row[u] * K + col[u]) = quant8<FMT, SF>(v[u], sc);
-        if (hl == 0) s[row[u] * ng + (col[u] >> 7)] = sc.s;
+      if (item_ok[u]) {
+        uint8_t* dst = q + row[u] * K + col[u];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (col[u] + 16 * h < K) {
+            const uint2 lo = quant8<FMT, SF>(v[u][2 * h], sc);
+            const uint2 hi = quant8<FMT, SF>(v[u][2 * h + 1], sc);
+            *reinterpret_cast<uint4*>(dst + 16 * h) = make_uint4(lo.x, lo.y, hi.x, hi.y);
+          }
+        }
+        if (qt == 0) s[row[u] * ng + (col[u] >> 7)] = sc.s;
       }
     }
   }
