@@ -48,7 +48,7 @@ def load_peaks():
 
 def source_sha() -> str:
     h = hashlib.sha256()
-    for f in ("gemm.cuh", "ptx.cuh", "quant.cuh", "fp8lin.cu"):
+    for f in ("gemm.cuh", "gemm_swap.cuh", "ptx.cuh", "quant.cuh", "fp8lin.cu"):
         h.update(open(os.path.join(ROOT, "fp8_block_scaled_12_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 

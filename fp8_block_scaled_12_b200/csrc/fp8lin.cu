@@ -9,6 +9,7 @@
 
 #include "../../include/fp8lin.h"
 #include "gemm.cuh"
+#include "gemm_swap.cuh"
 #include "ptx.cuh"
 #include "quant.cuh"
 
@@ -84,20 +85,21 @@ bool launch_regs_ok(K kern) {
   return fa.numRegs == int(kLaunchRegs);
 }
 
-template <int NT, int STAGES>
+template <int NT, int NBUF, int STAGES, int KB_CAP>
 int launch_swap(const void* qa, const void* qw, const GemmArgs& a, int64_t w_rows, cudaStream_t st) {
-  using C = SwapCfg<NT, STAGES>;
+  using C = SwapCfg<NT, NBUF, STAGES, KB_CAP>;
+  constexpr size_t smem = swap_smem_bytes<C>();
   CUtensorMap mw, mx;
   if (!make_map_u8(&mw, qw, uint64_t(w_rows), uint64_t(a.K), 128)) return FP8_ERR_CUDA;
   if (!make_map_u8(&mx, qa, uint64_t(a.M > 0 ? a.M : 1), uint64_t(a.K), 32)) return FP8_ERR_CUDA;
-  auto kern = k_gemm_swap<NT, STAGES>;
+  auto kern = k_gemm_swap<NT, NBUF, STAGES, KB_CAP>;
   if (!launch_regs_ok(kern)) return FP8_ERR_UNSUPPORTED;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(C::SMEM));
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return FP8_ERR_CUDA;
   const int nbn = (a.N + 127) / 128;
   const int64_t units = int64_t(a.E) * nbn;
   const int grid = int(units < num_sms() ? units : num_sms());
-  kern<<<grid, kThreads, C::SMEM, st>>>(mw, mx, a);
+  kern<<<grid, kThreads, smem, st>>>(mw, mx, a);
   return cuda_status(cudaGetLastError());
 }
 
@@ -242,9 +244,8 @@ int fp8_block_gemm(const void* qa, const float* sa, const void* qw, const float*
   if (M == 0) return FP8_OK;
   GemmArgs a{sa, sw, y, nullptr, int(M), int(N), int(K), 1, out_dtype == FP8_OUT_FP32 ? 1 : 0};
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (M <= 64) return launch_swap<64, 8>(qa, qw, a, N, st);
-  if (M <= 128) return launch_swap<128, 6>(qa, qw, a, N, st);
-  if (M <= 256) return launch_swap<256, 4>(qa, qw, a, N, st);
+  if (M <= 64) return launch_swap<64, 4, 7, 96>(qa, qw, a, N, st);
+  if (M <= 160) return launch_swap<160, 3, 4, 80>(qa, qw, a, N, st);
   return launch_wide(qa, qw, a, st);
 }
 
@@ -259,7 +260,7 @@ int fp8_grouped_gemm(const void* qa, const float* sa, const void* qw, const floa
   if (total_M == 0) return FP8_OK;
   GemmArgs a{sa, sw, y, group_offsets, int(total_M), int(N), int(K), int(E),
              out_dtype == FP8_OUT_FP32 ? 1 : 0};
-  return launch_swap<256, 4>(qa, qw, a, E * N, static_cast<cudaStream_t>(stream));
+  return launch_swap<160, 3, 4, 80>(qa, qw, a, E * N, static_cast<cudaStream_t>(stream));
 }
 
 int fp8_device_error(void* stream) {

@@ -23,9 +23,8 @@
 //
 //   k_gemm_wide   M-side = 128 activation rows, N-side = 256 weight rows per tile;
 //                 persistent over tiles, M fastest so concurrent CTAs share weights.
-//   k_gemm_swap   M-side = 128 weight rows, N-side = up to NT tokens: for decode
-//                 (few tokens) and for the grouped MoE GEMM, where the MMA's N is set
-//                 per tile to the expert's token count rounded up to 16.
+//   (gemm_swap.cuh holds the weight-stationary variant used for few tokens and for
+//   the grouped MoE GEMM.)
 #pragma once
 
 #include <cstdint>
@@ -255,237 +254,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             v[2 * t + 1] = f.y;
           }
           if (n0 + j < args.N) store8(args.y, out32, m * args.N + n0 + j, v);
-        }
-      }
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (*abort) {
-    if (threadIdx.x == 0) settle_ns(200000);
-    __syncthreads();
-  }
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, C::TMEM_COLS);
-  }
-}
-
-// =====================================================================
-// Swap kernel: tile = 128 weight rows x up to NT tokens (one expert's rows).
-// =====================================================================
-template <int NT, int STAGES>
-struct SwapCfg {
-  static constexpr uint32_t W_BYTES = 128 * kTileBytesPerRow;      // 16 KB
-  static constexpr uint32_t X_BYTES = NT * kTileBytesPerRow;
-  static constexpr uint32_t STAGE_BYTES = W_BYTES + X_BYTES;
-  static constexpr uint32_t TMEM_COLS = (2 * NT < 32) ? 32 : 2 * NT;
-  static constexpr int COLS_PER_WG = NT / 2;                       // token columns per warpgroup
-  static constexpr size_t CS_BYTES = 2 * NT * sizeof(float);   // [slot][NT] column scales
-  static constexpr size_t SMEM = 1024 + size_t(STAGES) * STAGE_BYTES + CS_BYTES + sizeof(PipeState<STAGES>);
-};
-
-// Unit u -> (expert, weight row-block); units of one expert are consecutive so the
-// expert's token rows are re-read from L2 while its weights stream from HBM once.
-__device__ __forceinline__ void group_range(const GemmArgs& a, int e, int& r0, int& r1) {
-  if (a.offsets == nullptr) {
-    r0 = 0;
-    r1 = a.M;
-  } else {
-    r0 = __ldg(a.offsets + e);
-    r1 = __ldg(a.offsets + e + 1);
-    r1 = min(r1, a.M);
-    r0 = min(r0, r1);
-  }
-}
-
-template <int NT, int STAGES>
-__global__ void __launch_bounds__(kThreads, 1)
-    k_gemm_swap(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
-                const GemmArgs args) {
-  using C = SwapCfg<NT, STAGES>;
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw = smem_u32(smem_raw);
-  const uint32_t base = (raw + 1023u) & ~1023u;
-  uint8_t* gbase = smem_raw + (base - raw);
-  float* colscale = reinterpret_cast<float*>(gbase + size_t(STAGES) * C::STAGE_BYTES);
-  PipeState<STAGES>* ps =
-      reinterpret_cast<PipeState<STAGES>*>(gbase + size_t(STAGES) * C::STAGE_BYTES + C::CS_BYTES);
-  volatile int* abort = &ps->abort;
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nbn = (args.N + 127) / 128;
-  const int num_units = args.E * nbn;
-  const int nkb = args.K / kBK;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(smem_u32(&ps->full[s]), 1);
-      mbar_init(smem_u32(&ps->empty[s]), 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(smem_u32(&ps->tfull[b]), 1);
-      mbar_init(smem_u32(&ps->tempty[b]), kEpiThreads / 32);
-      mbar_init(smem_u32(&ps->csfull[0][b]), 4);
-      mbar_init(smem_u32(&ps->csfull[1][b]), 4);
-    }
-    ps->abort = 0;
-    fence_barrier_init();
-    tma_prefetch_desc(&tmW);
-    tma_prefetch_desc(&tmX);
-  }
-  if (warp == 1) {
-    tmem_alloc(smem_u32(&ps->tmem_base), C::TMEM_COLS);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = ps->tmem_base;
-
-  if (warp < 4) {
-    setmaxnreg_dec<kProducerRegs>();
-    if (warp == 0 && lane == 0) {
-      // ------------------------------------------------ TMA producer
-      uint32_t it = 0;
-      for (int u = blockIdx.x; u < num_units && !*abort; u += gridDim.x) {
-        const int e = u / nbn, nb = u % nbn;
-        int r0, r1;
-        group_range(args, e, r0, r1);
-        for (int c0 = r0; c0 < r1 && !*abort; c0 += NT) {
-          const int cnt = min(NT, r1 - c0);
-          const int nbox = (cnt + 31) / 32;
-          for (int kb = 0; kb < nkb; ++kb, ++it) {
-            const int s = it % STAGES;
-            const uint32_t ph = (it / STAGES) & 1u;
-            if (!mbar_wait(smem_u32(&ps->empty[s]), ph ^ 1u, abort)) break;
-            const uint32_t w_addr = base + s * C::STAGE_BYTES;
-            const uint32_t bar = smem_u32(&ps->full[s]);
-            mbar_arrive_expect_tx(bar, C::W_BYTES + uint32_t(nbox) * 32u * kTileBytesPerRow);
-            tma_load_2d(w_addr, &tmW, bar, kb * kBK, e * args.N + nb * 128);
-            for (int i = 0; i < nbox; ++i)
-              tma_load_2d(w_addr + C::W_BYTES + i * 32 * kTileBytesPerRow, &tmX, bar, kb * kBK,
-                          c0 + 32 * i);
-          }
-        }
-      }
-    } else if (warp == 1 && lane == 0) {
-      // ------------------------------------------------ MMA issuer
-      uint32_t it = 0, kbc = 0;
-      for (int u = blockIdx.x; u < num_units && !*abort; u += gridDim.x) {
-        const int e = u / nbn;
-        int r0, r1;
-        group_range(args, e, r0, r1);
-        for (int c0 = r0; c0 < r1 && !*abort; c0 += NT) {
-          const int cnt = min(NT, r1 - c0);
-          const uint32_t n_mma = uint32_t((cnt + 15) / 16 * 16);
-          const uint32_t idesc = idesc_f8_e4m3_f32(128, n_mma);
-          for (int kb = 0; kb < nkb; ++kb, ++it, ++kbc) {
-            const int s = it % STAGES;
-            const uint32_t ph = (it / STAGES) & 1u;
-            const uint32_t b = kbc & 1u;
-            if (!mbar_wait(smem_u32(&ps->tempty[b]), ((kbc >> 1) & 1u) ^ 1u, abort)) break;
-            if (!mbar_wait(smem_u32(&ps->full[s]), ph, abort)) break;
-            tc_fence_after();
-            const uint32_t w_addr = base + s * C::STAGE_BYTES;
-            const uint32_t x_addr = w_addr + C::W_BYTES;
-            const uint32_t d = tmem + b * NT;
-#pragma unroll
-            for (int k = 0; k < kBK / 32; ++k)
-              mma_f8(d, sw128_kmajor_desc(w_addr + k * 32), sw128_kmajor_desc(x_addr + k * 32), idesc,
-                     k > 0 ? 1u : 0u);
-            mma_commit(smem_u32(&ps->empty[s]));
-            mma_commit(smem_u32(&ps->tfull[b]));
-          }
-        }
-      }
-    }
-  } else {
-    setmaxnreg_inc<kConsumerRegs>();
-    // ------------------------------------------------ promotion + epilogue
-    constexpr int CW = C::COLS_PER_WG;
-    const int ew = threadIdx.x - 128;    // 0..255
-    const int wg = ew >> 7;              // token-column half
-    const int t_in_wg = ew & 127;
-    const int quad = warp & 3;
-    const bool out32 = args.out_fp32 != 0;
-    float* cs = colscale + wg * CW;      // slot p of this warpgroup: cs[p * NT + j]
-    // Column scales move from the threads that load them to all threads of the
-    // warpgroup through a 2-slot ring guarded by mbarriers (4 warp arrivals per
-    // fill).  Slot kbc & 1 holds K-block kbc's scales; a thread only refills a slot
-    // after passing the wait for the other slot, which every thread arrives on only
-    // after it has finished reading this slot's previous contents.
-    uint32_t kbc = 0;
-    bool aborted = false;
-    for (int u = blockIdx.x; u < num_units && !aborted; u += gridDim.x) {
-      const int e = u / nbn, nb = u % nbn;
-      const int n = nb * 128 + quad * 32 + lane;        // weight row of this thread
-      const bool n_ok = n < args.N;
-      const float* sw_blk = args.sw + (int64_t(e) * nbn + nb) * nkb;
-      int r0, r1;
-      group_range(args, e, r0, r1);
-      for (int c0 = r0; c0 < r1; c0 += NT) {
-        const int cnt = min(NT, r1 - c0);
-        const int col0 = wg * CW;                       // first token column of this WG
-        // this thread loads the scale of token (c0 + col0 + t_in_wg), times sw[kb]
-        const bool tok_ok = (t_in_wg < CW) && (col0 + t_in_wg < cnt);
-        const float* sa_tok = args.sa + int64_t(tok_ok ? c0 + col0 + t_in_wg : 0) * nkb;
-        if (t_in_wg < CW) cs[(kbc & 1u) * NT + t_in_wg] = tok_ok ? __ldg(sa_tok) * __ldg(sw_blk) : 0.0f;
-        float next = (tok_ok && nkb > 1) ? __ldg(sa_tok + 1) * __ldg(sw_blk + 1) : 0.0f;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&ps->csfull[wg][kbc & 1u]));
-        uint64_t acc[CW / 2];              // CW fp32 accumulators as packed pairs
-#pragma unroll
-        for (int j = 0; j < CW / 2; ++j) acc[j] = 0ull;
-        for (int kb = 0; kb < nkb; ++kb, ++kbc) {
-          const uint32_t b = kbc & 1u;
-          if (!mbar_wait(smem_u32(&ps->csfull[wg][b]), (kbc >> 1) & 1u, abort)) { aborted = true; break; }
-          if (!mbar_wait(smem_u32(&ps->tfull[b]), (kbc >> 1) & 1u, abort)) { aborted = true; break; }
-          tc_fence_after();
-          const float* csk = cs + b * NT;
-          const uint32_t taddr = tmem + (uint32_t(quad * 32) << 16) + b * NT + col0;
-#pragma unroll
-          for (int h = 0; h < CW / 32; ++h) {
-            uint32_t p[32];
-            tmem_ld32(taddr + h * 32, p);
-            tmem_ld_wait();
-            if (h == CW / 32 - 1) {
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(smem_u32(&ps->tempty[b]));
-            }
-#pragma unroll
-            for (int j = 0; j < 32; j += 4) {
-              const ulonglong2 sc = *reinterpret_cast<const ulonglong2*>(csk + h * 32 + j);
-              ffma2(acc[(h * 32 + j) / 2], p[j], p[j + 1], sc.x);
-              ffma2(acc[(h * 32 + j) / 2 + 1], p[j + 2], p[j + 3], sc.y);
-            }
-          }
-          // fill the other slot with K-block kb+1's column scales
-          if (kb + 1 < nkb) {
-            if (t_in_wg < CW) cs[(b ^ 1u) * NT + t_in_wg] = next;
-            if (kb + 2 < nkb) next = tok_ok ? __ldg(sa_tok + kb + 2) * __ldg(sw_blk + kb + 2) : 0.0f;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&ps->csfull[wg][b ^ 1u]));
-          }
-        }
-        if (aborted) break;
-        if (n_ok) {
-          const int jmax = min(CW, cnt - col0);
-          const int64_t idx0 = int64_t(c0 + col0) * args.N + n;
-#pragma unroll
-          for (int j = 0; j < CW; ++j) {
-            if (j < jmax) {
-              const int64_t idx = idx0 + int64_t(j) * args.N;
-              const float2 f = unpack2(acc[j / 2]);
-              const float v = (j & 1) ? f.y : f.x;
-              if (out32)
-                reinterpret_cast<float*>(args.y)[idx] = v;
-              else
-                reinterpret_cast<__nv_bfloat16*>(args.y)[idx] = __float2bfloat16_rn(v);
-            }
-          }
         }
       }
     }

@@ -1,0 +1,307 @@
+// gemm_swap.cuh -- weight-stationary block-scaled FP8 GEMM for few tokens per weight
+// tile: decode (M <= 160) and the grouped MoE expert GEMM.
+//
+// Same operation as gemm.cuh ("FP8 推理提速 83.6%: DeepSeek-V3 在 AMD MI250 上的完整落地
+// 指南", 运行时: fp8_gemm; MoE: 256 routed experts, 8 active per token), with the
+// operands swapped on the tensor core: the MMA's M side is 128 weight rows and its N
+// side is up to NT tokens, so a handful of tokens still fills the 128-row datapath and
+// each weight byte is streamed from HBM once.  A work unit is (expert e, weight
+// row-block nb); units of one expert are consecutive, so the expert's token rows are
+// re-read from L2 while its weights stream from HBM.  Per unit the expert's rows are
+// taken in chunks of at most NT tokens and the MMA's N is set per chunk to the token
+// count rounded up to 16 (the instruction descriptor is a runtime value).
+//
+// Roles (384 threads):
+//   warp 0       TMA producer: weight tile (128 rows x 128 K) plus the chunk's token
+//                rows in 32-row boxes per K-block stage.
+//   warps 1-3    MMA issuers, taking K-blocks round robin.  A thread's own barrier
+//                waits stall until the MMAs it issued before them finish, so a single
+//                issuer leaves the tensor pipe idle around every wait; with three, the
+//                others' MMAs keep it busy.  K-blocks use separate stages and buffers,
+//                so their order on the pipe does not matter.
+//   warps 4-11   promotion / epilogue: thread = one weight row (tensor-memory lane),
+//                warpgroup h = token columns [h*NT/2, (h+1)*NT/2).  Per K-block it loads
+//                all its columns in one batch, releases the buffer, then multiplies by
+//                sw[e][nb][kb] * sa[token][kb] (per column, from a table the warpgroup
+//                loads into shared memory once per chunk) and accumulates in fp32
+//                registers.
+#pragma once
+
+#include "gemm.cuh"
+
+namespace fp8lin {
+
+template <int NT_, int NBUF_, int STAGES_, int KB_CAP_>
+struct SwapCfg {
+  static constexpr int NT = NT_, NBUF = NBUF_, STAGES = STAGES_;
+  static constexpr int KB_CAP = KB_CAP_;                            // K-blocks per scale-table segment
+  static constexpr int CW = NT / 2;                                 // token columns per warpgroup
+  static constexpr uint32_t W_BYTES = 128 * kTileBytesPerRow;      // 16 KB
+  static constexpr uint32_t X_BYTES = NT * kTileBytesPerRow;
+  static constexpr uint32_t STAGE_BYTES = W_BYTES + X_BYTES;
+  static constexpr uint32_t TMEM_COLS = (NBUF * NT <= 32) ? 32 : (NBUF * NT <= 64) ? 64
+                                        : (NBUF * NT <= 128) ? 128 : (NBUF * NT <= 256) ? 256 : 512;
+  // per warpgroup: [KB_CAP][CW] column scales sa[token][kb] * sw[kb]
+  static constexpr size_t CS_BYTES = size_t(2) * KB_CAP * CW * sizeof(float);
+  static_assert(NT % 32 == 0 && NT <= 256, "token tile");
+  static_assert(NBUF * NT <= 512, "tensor memory holds 512 columns");
+  static_assert(CW % 16 == 0 && CW <= 96, "one-batch promotion needs CW staging registers");
+  static_assert(X_BYTES % 1024 == 0, "stages stay 1024-byte aligned");
+};
+
+template <int STAGES, int NBUF>
+struct alignas(8) SwapState {
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t tfull[NBUF];
+  uint64_t tempty[NBUF];
+  uint64_t tbl[2];         // per warpgroup: scale-table segment done reading / loaded
+  uint32_t tmem_base;
+  int abort;
+};
+
+template <class C>
+constexpr size_t swap_smem_bytes() {
+  return 1024 + size_t(C::STAGES) * C::STAGE_BYTES + C::CS_BYTES + sizeof(SwapState<C::STAGES, C::NBUF>);
+}
+
+// Rows of expert e: [r0, r1).  offsets == nullptr means one group [0, M).
+__device__ __forceinline__ void group_range(const GemmArgs& a, int e, int& r0, int& r1) {
+  if (a.offsets == nullptr) {
+    r0 = 0;
+    r1 = a.M;
+  } else {
+    r0 = __ldg(a.offsets + e);
+    r1 = __ldg(a.offsets + e + 1);
+    r1 = min(r1, a.M);
+    r0 = min(r0, r1);
+  }
+}
+
+constexpr int kSwapIssuers = 3;
+
+template <int NT, int NBUF, int STAGES, int KB_CAP>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_gemm_swap(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                const GemmArgs args) {
+  using C = SwapCfg<NT, NBUF, STAGES, KB_CAP>;
+  constexpr int CW = C::CW;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  float* colscale = reinterpret_cast<float*>(gbase + size_t(STAGES) * C::STAGE_BYTES);
+  auto* ps = reinterpret_cast<SwapState<STAGES, NBUF>*>(gbase + size_t(STAGES) * C::STAGE_BYTES + C::CS_BYTES);
+  volatile int* abort = &ps->abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nbn = (args.N + 127) / 128;
+  const int num_units = args.E * nbn;
+  const int nkb = args.K / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(&ps->full[s]), 1);
+      mbar_init(smem_u32(&ps->empty[s]), 1);
+    }
+    for (int b = 0; b < NBUF; ++b) {
+      mbar_init(smem_u32(&ps->tfull[b]), 1);
+      mbar_init(smem_u32(&ps->tempty[b]), kEpiThreads / 32);
+    }
+    mbar_init(smem_u32(&ps->tbl[0]), 4);
+    mbar_init(smem_u32(&ps->tbl[1]), 4);
+    ps->abort = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmW);
+    tma_prefetch_desc(&tmX);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&ps->tmem_base), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ps->tmem_base;
+
+  if (warp < 4) {
+    setmaxnreg_dec<kProducerRegs>();
+    if (warp == 0 && lane == 0) {
+      // ------------------------------------------------ TMA producer
+      uint32_t it = 0;
+      for (int u = blockIdx.x; u < num_units && !*abort; u += gridDim.x) {
+        const int e = u / nbn, nb = u % nbn;
+        int r0, r1;
+        group_range(args, e, r0, r1);
+        for (int c0 = r0; c0 < r1 && !*abort; c0 += NT) {
+          const int cnt = min(NT, r1 - c0);
+          const int nbox = (cnt + 31) / 32;
+          for (int kb = 0; kb < nkb; ++kb, ++it) {
+            const int s = it % STAGES;
+            const uint32_t ph = (it / STAGES) & 1u;
+            if (!mbar_wait(smem_u32(&ps->empty[s]), ph ^ 1u, abort)) break;
+            const uint32_t w_addr = base + s * C::STAGE_BYTES;
+            const uint32_t bar = smem_u32(&ps->full[s]);
+            mbar_arrive_expect_tx(bar, C::W_BYTES + uint32_t(nbox) * 32u * kTileBytesPerRow);
+            tma_load_2d(w_addr, &tmW, bar, kb * kBK, e * args.N + nb * 128);
+            for (int i = 0; i < nbox; ++i)
+              tma_load_2d(w_addr + C::W_BYTES + i * 32 * kTileBytesPerRow, &tmX, bar, kb * kBK, c0 + 32 * i);
+          }
+        }
+      }
+    } else if (warp >= 1 && warp <= kSwapIssuers && lane == 0) {
+      // ------------------------------------------------ MMA issuers (round robin over K-blocks)
+      const uint32_t mine = uint32_t(warp - 1);
+      uint32_t it = 0;
+      bool stop = false;
+      for (int u = blockIdx.x; u < num_units && !stop; u += gridDim.x) {
+        const int e = u / nbn;
+        int r0, r1;
+        group_range(args, e, r0, r1);
+        for (int c0 = r0; c0 < r1 && !stop; c0 += NT) {
+          const int cnt = min(NT, r1 - c0);
+          const uint32_t idesc = idesc_f8_e4m3_f32(128, uint32_t((cnt + 15) / 16 * 16));
+          for (int kb = 0; kb < nkb; ++kb, ++it) {
+            if (it % kSwapIssuers != mine) continue;
+            const int s = it % STAGES;
+            const uint32_t ph = (it / STAGES) & 1u;
+            const uint32_t b = it % NBUF;
+            if (!mbar_wait(smem_u32(&ps->tempty[b]), ((it / NBUF) & 1u) ^ 1u, abort)) { stop = true; break; }
+            if (!mbar_wait(smem_u32(&ps->full[s]), ph, abort)) { stop = true; break; }
+            tc_fence_after();
+            const uint32_t w_addr = base + s * C::STAGE_BYTES;
+            const uint32_t x_addr = w_addr + C::W_BYTES;
+            const uint32_t d = tmem + b * NT;
+#pragma unroll
+            for (int k = 0; k < kBK / 32; ++k)
+              mma_f8(d, sw128_kmajor_desc(w_addr + k * 32), sw128_kmajor_desc(x_addr + k * 32), idesc,
+                     k > 0 ? 1u : 0u);
+            mma_commit(smem_u32(&ps->empty[s]));
+            mma_commit(smem_u32(&ps->tfull[b]));
+          }
+        }
+      }
+    }
+  } else {
+    setmaxnreg_inc<kConsumerRegs>();
+    // ------------------------------------------------ promotion + epilogue
+    const int ew = threadIdx.x - 128;    // 0..255
+    const int wg = ew >> 7;              // token-column half
+    const int t_in_wg = ew & 127;
+    const int quad = warp & 3;
+    const bool out32 = args.out_fp32 != 0;
+    // This warpgroup's column-scale table: tbl[kb - seg0][j] = sa[token j][kb] * sw[kb]
+    // for a segment of up to KB_CAP K-blocks, loaded by all 128 threads at once (the
+    // reads are independent, so their latency overlaps) instead of one K-block at a
+    // time inside the promotion loop.  Each segment is bracketed by two phases of the
+    // warpgroup's mbarrier: "everyone finished reading the previous segment" and
+    // "the new segment is loaded".
+    float* table = colscale + size_t(wg) * KB_CAP * CW;
+    const uint32_t tbar = smem_u32(&ps->tbl[wg]);
+    uint32_t tphase = 0;
+    uint32_t kbc = 0;
+    bool aborted = false;
+    for (int u = blockIdx.x; u < num_units && !aborted; u += gridDim.x) {
+      const int e = u / nbn, nb = u % nbn;
+      const int n = nb * 128 + quad * 32 + lane;        // weight row of this thread
+      const bool n_ok = n < args.N;
+      const float* sw_blk = args.sw + (int64_t(e) * nbn + nb) * nkb;
+      int r0, r1;
+      group_range(args, e, r0, r1);
+      for (int c0 = r0; c0 < r1 && !aborted; c0 += NT) {
+        const int cnt = min(NT, r1 - c0);
+        const int col0 = wg * CW;                       // first token column of this WG
+        const int ncols = max(0, min(CW, cnt - col0));  // valid token columns of this WG
+        uint64_t acc[CW / 2];                            // CW fp32 accumulators as packed pairs
+#pragma unroll
+        for (int j = 0; j < CW / 2; ++j) acc[j] = 0ull;
+        for (int seg0 = 0; seg0 < nkb && !aborted; seg0 += KB_CAP) {
+          const int seglen = min(KB_CAP, nkb - seg0);
+          // phase 1: every thread of the warpgroup is done with the previous segment
+          __syncwarp();
+          if (lane == 0) mbar_arrive(tbar);
+          if (!mbar_wait(tbar, tphase & 1u, abort)) { aborted = true; break; }
+          ++tphase;
+          // load: entry (kb, j) for kb < seglen, j < CW (zeros for missing tokens).
+          // Batches of TB independent global loads go to registers first and are then
+          // stored, so their latencies overlap (a store between loads would order them).
+          constexpr int TB = 8;
+          const int total = seglen * CW;
+          for (int i0 = t_in_wg; i0 < total; i0 += 128 * TB) {
+            float v[TB];
+#pragma unroll
+            for (int q = 0; q < TB; ++q) {
+              const int i = i0 + 128 * q;
+              const int j = i / seglen, kk = i - j * seglen;   // consecutive threads walk a token's row
+              v[q] = (i < total && j < ncols)
+                         ? __ldg(args.sa + int64_t(c0 + col0 + j) * nkb + seg0 + kk) * __ldg(sw_blk + seg0 + kk)
+                         : 0.0f;
+            }
+#pragma unroll
+            for (int q = 0; q < TB; ++q) {
+              const int i = i0 + 128 * q;
+              const int j = i / seglen, kk = i - j * seglen;
+              if (i < total) table[kk * CW + j] = v[q];
+            }
+          }
+          // phase 2: the segment is loaded
+          __syncwarp();
+          if (lane == 0) mbar_arrive(tbar);
+          if (!mbar_wait(tbar, tphase & 1u, abort)) { aborted = true; break; }
+          ++tphase;
+          for (int kk = 0; kk < seglen; ++kk, ++kbc) {
+            const uint32_t b = kbc % NBUF;
+            if (!mbar_wait(smem_u32(&ps->tfull[b]), (kbc / NBUF) & 1u, abort)) { aborted = true; break; }
+            tc_fence_after();
+            const uint32_t taddr = tmem + (uint32_t(quad * 32) << 16) + b * NT + col0;
+            uint32_t p[CW];
+#pragma unroll
+            for (int c = 0; c + 32 <= CW; c += 32) tmem_ld32(taddr + c, *reinterpret_cast<uint32_t(*)[32]>(&p[c]));
+            if constexpr (CW % 32 == 16)
+              tmem_ld16(taddr + (CW - 16), *reinterpret_cast<uint32_t(*)[16]>(&p[CW - 16]));
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&ps->tempty[b]));
+            const float* csk = table + kk * CW;
+#pragma unroll
+            for (int j = 0; j < CW; j += 4) {
+              const ulonglong2 sc = *reinterpret_cast<const ulonglong2*>(csk + j);
+              ffma2(acc[j / 2], p[j], p[j + 1], sc.x);
+              ffma2(acc[j / 2 + 1], p[j + 2], p[j + 3], sc.y);
+            }
+          }
+        }
+        if (aborted) break;
+        if (n_ok) {
+          const int64_t idx0 = int64_t(c0 + col0) * args.N + n;
+#pragma unroll
+          for (int j = 0; j < CW; ++j) {
+            if (j < ncols) {
+              const int64_t idx = idx0 + int64_t(j) * args.N;
+              const float2 f = unpack2(acc[j / 2]);
+              const float v = (j & 1) ? f.y : f.x;
+              if (out32)
+                reinterpret_cast<float*>(args.y)[idx] = v;
+              else
+                reinterpret_cast<__nv_bfloat16*>(args.y)[idx] = __float2bfloat16_rn(v);
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (*abort) {
+    if (threadIdx.x == 0) settle_ns(200000);
+    __syncthreads();
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace fp8lin

@@ -69,9 +69,9 @@ def test_tiny_config(cuda_device):
     gemm_and_compare(cuda_device, p["M"], p["N"], p["K"], outliers=p["outliers"], factor=p["factor"])
 
 
-@pytest.mark.parametrize("M", [1, 8, 16, 40, 64, 65, 100, 128, 200, 256])
+@pytest.mark.parametrize("M", [1, 8, 16, 40, 64, 65, 100, 128, 150, 160, 161, 200, 256])
 def test_swap_path_token_counts(cuda_device, M):
-    """M <= 256 runs the weight-stationary kernel; ragged token counts, N and K span
+    """M <= 160 runs the weight-stationary kernel, larger M the 128x256 tile kernel; ragged token counts, N and K span
     several tiles."""
     gemm_and_compare(cuda_device, M, 384, 1024, seed=M)
 
