@@ -244,8 +244,8 @@ int fp8_block_gemm(const void* qa, const float* sa, const void* qw, const float*
   if (M == 0) return FP8_OK;
   GemmArgs a{sa, sw, y, nullptr, int(M), int(N), int(K), 1, out_dtype == FP8_OUT_FP32 ? 1 : 0};
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (M <= 64) return launch_swap<64, 4, 7, 96>(qa, qw, a, N, st);
-  if (M <= 160) return launch_swap<160, 3, 4, 80>(qa, qw, a, N, st);
+  if (M <= 64) return launch_swap<64, 4, 8, 56>(qa, qw, a, N, st);
+  if (M <= 160) return launch_swap<160, 3, 5, 28>(qa, qw, a, N, st);
   return launch_wide(qa, qw, a, st);
 }
 
@@ -260,7 +260,7 @@ int fp8_grouped_gemm(const void* qa, const float* sa, const void* qw, const floa
   if (total_M == 0) return FP8_OK;
   GemmArgs a{sa, sw, y, group_offsets, int(total_M), int(N), int(K), int(E),
              out_dtype == FP8_OUT_FP32 ? 1 : 0};
-  return launch_swap<160, 3, 4, 80>(qa, qw, a, E * N, static_cast<cudaStream_t>(stream));
+  return launch_swap<160, 3, 5, 28>(qa, qw, a, E * N, static_cast<cudaStream_t>(stream));
 }
 
 int fp8_device_error(void* stream) {

@@ -22,9 +22,15 @@
 //   warps 4-11   promotion / epilogue: thread = one weight row (tensor-memory lane),
 //                warpgroup h = token columns [h*NT/2, (h+1)*NT/2).  Per K-block it loads
 //                all its columns in one batch, releases the buffer, then multiplies by
-//                sw[e][nb][kb] * sa[token][kb] (per column, from a table the warpgroup
-//                loads into shared memory once per chunk) and accumulates in fp32
-//                registers.
+//                sw * sa[token] and accumulates in fp32 registers.
+//
+// Scales.  The work of a CTA is a sequence of segments (unit, token chunk, up to
+// KB_CAP K-blocks).  A segment's scales -- sa[token][kb] for the chunk's tokens and
+// sw[e][nb][kb] -- sit in one of two shared-memory tables, row kb holding the tokens
+// side by side so the promotion reads four columns per 16-byte load.  The epilogue
+// threads fill the table of the NEXT segment with 4-byte cp.async while they promote
+// the current one, so only the first segment's load is exposed.  The chunk's sa rows
+// are consecutive in memory, so each warp's copies read 128 contiguous bytes.
 #pragma once
 
 #include "gemm.cuh"
@@ -34,19 +40,20 @@ namespace fp8lin {
 template <int NT_, int NBUF_, int STAGES_, int KB_CAP_>
 struct SwapCfg {
   static constexpr int NT = NT_, NBUF = NBUF_, STAGES = STAGES_;
-  static constexpr int KB_CAP = KB_CAP_;                            // K-blocks per scale-table segment
+  static constexpr int KB_CAP = KB_CAP_;                            // K-blocks per segment
   static constexpr int CW = NT / 2;                                 // token columns per warpgroup
+  static constexpr int TROW = NT + 4;                               // table row: sa[0..NT), sw at [NT]
+  static constexpr uint32_t TBUF_BYTES = uint32_t(KB_CAP) * TROW * 4;
   static constexpr uint32_t W_BYTES = 128 * kTileBytesPerRow;      // 16 KB
   static constexpr uint32_t X_BYTES = NT * kTileBytesPerRow;
   static constexpr uint32_t STAGE_BYTES = W_BYTES + X_BYTES;
   static constexpr uint32_t TMEM_COLS = (NBUF * NT <= 32) ? 32 : (NBUF * NT <= 64) ? 64
                                         : (NBUF * NT <= 128) ? 128 : (NBUF * NT <= 256) ? 256 : 512;
-  // per warpgroup: [KB_CAP][CW] column scales sa[token][kb] * sw[kb]
-  static constexpr size_t CS_BYTES = size_t(2) * KB_CAP * CW * sizeof(float);
   static_assert(NT % 32 == 0 && NT <= 256, "token tile");
   static_assert(NBUF * NT <= 512, "tensor memory holds 512 columns");
   static_assert(CW % 16 == 0 && CW <= 96, "one-batch promotion needs CW staging registers");
   static_assert(X_BYTES % 1024 == 0, "stages stay 1024-byte aligned");
+  static_assert(TBUF_BYTES % 16 == 0, "table rows keep 16-byte alignment");
 };
 
 template <int STAGES, int NBUF>
@@ -55,14 +62,14 @@ struct alignas(8) SwapState {
   uint64_t empty[STAGES];
   uint64_t tfull[NBUF];
   uint64_t tempty[NBUF];
-  uint64_t tbl[2];         // per warpgroup: scale-table segment done reading / loaded
+  uint64_t seg;            // epilogue warps: segment's table loaded, previous one retired
   uint32_t tmem_base;
   int abort;
 };
 
 template <class C>
 constexpr size_t swap_smem_bytes() {
-  return 1024 + size_t(C::STAGES) * C::STAGE_BYTES + C::CS_BYTES + sizeof(SwapState<C::STAGES, C::NBUF>);
+  return 1024 + size_t(C::STAGES) * C::STAGE_BYTES + 2 * size_t(C::TBUF_BYTES) + sizeof(SwapState<C::STAGES, C::NBUF>);
 }
 
 // Rows of expert e: [r0, r1).  offsets == nullptr means one group [0, M).
@@ -80,6 +87,54 @@ __device__ __forceinline__ void group_range(const GemmArgs& a, int e, int& r0, i
 
 constexpr int kSwapIssuers = 3;
 
+// One segment of a CTA's work: unit u (expert e = u / nbn, weight row-block
+// nb = u % nbn), token rows [c0, min(c0 + NT, r1)), K-blocks [seg0, seg0 + KB_CAP).
+struct SwapSeg {
+  int u, c0, r1, seg0;
+};
+
+// First segment of the first unit at or after u (in steps of gridDim.x) that has rows.
+__device__ __forceinline__ bool swap_seg_find(const GemmArgs& a, int nbn, int num_units, int u, SwapSeg& s) {
+  for (; u < num_units; u += gridDim.x) {
+    int r0, r1;
+    group_range(a, u / nbn, r0, r1);
+    if (r0 < r1) {
+      s = SwapSeg{u, r0, r1, 0};
+      return true;
+    }
+  }
+  return false;
+}
+
+// Advance to the next segment in the order the producer and the issuers walk
+// (K-blocks, then token chunks, then units).
+template <int NT, int KB_CAP>
+__device__ __forceinline__ bool swap_seg_next(const GemmArgs& a, int nbn, int num_units, int nkb, SwapSeg& s) {
+  s.seg0 += KB_CAP;
+  if (s.seg0 < nkb) return true;
+  s.seg0 = 0;
+  s.c0 += NT;
+  if (s.c0 < s.r1) return true;
+  return swap_seg_find(a, nbn, num_units, s.u + gridDim.x, s);
+}
+
+// All 256 epilogue threads: start the copies of segment s's scales into the table at
+// shared address `tbl`: row kk holds sa[c0 + j][seg0 + kk] at column j, sw at NT.
+template <class C>
+__device__ __forceinline__ void swap_seg_load(const GemmArgs& a, const SwapSeg& s, int nbn, int nkb, uint32_t tbl,
+                                              int ewarp, int lane) {
+  const int cnt = min(C::NT, s.r1 - s.c0);
+  const int seglen = min(C::KB_CAP, nkb - s.seg0);
+  const float* src = a.sa + int64_t(s.c0) * nkb + s.seg0;
+  for (int j = ewarp; j < cnt; j += kEpiThreads / 32)
+    for (int kk = lane; kk < seglen; kk += 32)
+      cp_async4(tbl + 4u * uint32_t(kk * C::TROW + j), src + int64_t(j) * nkb + kk);
+  if (ewarp == 0) {
+    const float* sws = a.sw + (int64_t(s.u / nbn) * nbn + s.u % nbn) * nkb + s.seg0;
+    for (int kk = lane; kk < seglen; kk += 32) cp_async4(tbl + 4u * uint32_t(kk * C::TROW + C::NT), sws + kk);
+  }
+}
+
 template <int NT, int NBUF, int STAGES, int KB_CAP>
 __global__ void __launch_bounds__(kThreads, 1)
     k_gemm_swap(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
@@ -90,8 +145,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (base - raw);
-  float* colscale = reinterpret_cast<float*>(gbase + size_t(STAGES) * C::STAGE_BYTES);
-  auto* ps = reinterpret_cast<SwapState<STAGES, NBUF>*>(gbase + size_t(STAGES) * C::STAGE_BYTES + C::CS_BYTES);
+  float* table = reinterpret_cast<float*>(gbase + size_t(STAGES) * C::STAGE_BYTES);
+  auto* ps = reinterpret_cast<SwapState<STAGES, NBUF>*>(gbase + size_t(STAGES) * C::STAGE_BYTES + 2 * size_t(C::TBUF_BYTES));
   volatile int* abort = &ps->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -108,8 +163,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&ps->tfull[b]), 1);
       mbar_init(smem_u32(&ps->tempty[b]), kEpiThreads / 32);
     }
-    mbar_init(smem_u32(&ps->tbl[0]), 4);
-    mbar_init(smem_u32(&ps->tbl[1]), 4);
+    mbar_init(smem_u32(&ps->seg), kEpiThreads / 32);
     ps->abort = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmW);
@@ -186,110 +240,86 @@ __global__ void __launch_bounds__(kThreads, 1)
     setmaxnreg_inc<kConsumerRegs>();
     // ------------------------------------------------ promotion + epilogue
     const int ew = threadIdx.x - 128;    // 0..255
+    const int ewarp = ew >> 5;           // 0..7
     const int wg = ew >> 7;              // token-column half
-    const int t_in_wg = ew & 127;
     const int quad = warp & 3;
     const bool out32 = args.out_fp32 != 0;
-    // This warpgroup's column-scale table: tbl[kb - seg0][j] = sa[token j][kb] * sw[kb]
-    // for a segment of up to KB_CAP K-blocks, loaded by all 128 threads at once (the
-    // reads are independent, so their latency overlaps) instead of one K-block at a
-    // time inside the promotion loop.  Each segment is bracketed by two phases of the
-    // warpgroup's mbarrier: "everyone finished reading the previous segment" and
-    // "the new segment is loaded".
-    float* table = colscale + size_t(wg) * KB_CAP * CW;
-    const uint32_t tbar = smem_u32(&ps->tbl[wg]);
-    uint32_t tphase = 0;
-    uint32_t kbc = 0;
+    const int col0 = wg * CW;            // first token column of this warpgroup
+    const uint32_t table_s = smem_u32(table);
+    const uint32_t segbar = smem_u32(&ps->seg);
+    SwapSeg cur;
+    bool have = swap_seg_find(args, nbn, num_units, blockIdx.x, cur);
+    if (have) swap_seg_load<C>(args, cur, nbn, nkb, table_s, ewarp, lane);
+    uint32_t sidx = 0, kbc = 0;
     bool aborted = false;
-    for (int u = blockIdx.x; u < num_units && !aborted; u += gridDim.x) {
-      const int e = u / nbn, nb = u % nbn;
-      const int n = nb * 128 + quad * 32 + lane;        // weight row of this thread
-      const bool n_ok = n < args.N;
-      const float* sw_blk = args.sw + (int64_t(e) * nbn + nb) * nkb;
-      int r0, r1;
-      group_range(args, e, r0, r1);
-      for (int c0 = r0; c0 < r1 && !aborted; c0 += NT) {
-        const int cnt = min(NT, r1 - c0);
-        const int col0 = wg * CW;                       // first token column of this WG
-        const int ncols = max(0, min(CW, cnt - col0));  // valid token columns of this WG
-        uint64_t acc[CW / 2];                            // CW fp32 accumulators as packed pairs
+    uint64_t acc[CW / 2];                                // CW fp32 accumulators as packed pairs
+    while (have) {
+      const int seglen = min(KB_CAP, nkb - cur.seg0);
+      if (cur.seg0 == 0) {
 #pragma unroll
         for (int j = 0; j < CW / 2; ++j) acc[j] = 0ull;
-        for (int seg0 = 0; seg0 < nkb && !aborted; seg0 += KB_CAP) {
-          const int seglen = min(KB_CAP, nkb - seg0);
-          // phase 1: every thread of the warpgroup is done with the previous segment
-          __syncwarp();
-          if (lane == 0) mbar_arrive(tbar);
-          if (!mbar_wait(tbar, tphase & 1u, abort)) { aborted = true; break; }
-          ++tphase;
-          // load: entry (kb, j) for kb < seglen, j < CW (zeros for missing tokens).
-          // Batches of TB independent global loads go to registers first and are then
-          // stored, so their latencies overlap (a store between loads would order them).
-          constexpr int TB = 8;
-          const int total = seglen * CW;
-          for (int i0 = t_in_wg; i0 < total; i0 += 128 * TB) {
-            float v[TB];
+      }
+      // This segment's table is complete once every warp has seen its own copies
+      // land; the same arrival says the warp is done with the previous segment, whose
+      // buffer the next prefetch overwrites.
+      cp_async_wait_all();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(segbar);
+      bool ok = mbar_wait(segbar, sidx & 1u, abort);
+      if (__any_sync(0xffffffffu, !ok)) { aborted = true; break; }
+      {
+        SwapSeg nxt = cur;
+        if (swap_seg_next<NT, KB_CAP>(args, nbn, num_units, nkb, nxt))
+          swap_seg_load<C>(args, nxt, nbn, nkb, table_s + ((sidx + 1) & 1u) * C::TBUF_BYTES, ewarp, lane);
+      }
+      const float* tb = table + (sidx & 1u) * (C::TBUF_BYTES / 4);
+      for (int kk = 0; kk < seglen; ++kk, ++kbc) {
+        const uint32_t b = kbc % NBUF;
+        ok = mbar_wait(smem_u32(&ps->tfull[b]), (kbc / NBUF) & 1u, abort);
+        if (__any_sync(0xffffffffu, !ok)) { aborted = true; break; }
+        tc_fence_after();
+        const uint32_t taddr = tmem + (uint32_t(quad * 32) << 16) + b * NT + col0;
+        uint32_t p[CW];
 #pragma unroll
-            for (int q = 0; q < TB; ++q) {
-              const int i = i0 + 128 * q;
-              const int j = i / seglen, kk = i - j * seglen;   // consecutive threads walk a token's row
-              v[q] = (i < total && j < ncols)
-                         ? __ldg(args.sa + int64_t(c0 + col0 + j) * nkb + seg0 + kk) * __ldg(sw_blk + seg0 + kk)
-                         : 0.0f;
-            }
+        for (int c = 0; c + 32 <= CW; c += 32) tmem_ld32(taddr + c, *reinterpret_cast<uint32_t(*)[32]>(&p[c]));
+        if constexpr (CW % 32 == 16)
+          tmem_ld16(taddr + (CW - 16), *reinterpret_cast<uint32_t(*)[16]>(&p[CW - 16]));
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&ps->tempty[b]));
+        const float* row = tb + kk * C::TROW;
+        const float swv = row[NT];
+        const uint64_t sw2 = pack2(swv, swv);
 #pragma unroll
-            for (int q = 0; q < TB; ++q) {
-              const int i = i0 + 128 * q;
-              const int j = i / seglen, kk = i - j * seglen;
-              if (i < total) table[kk * CW + j] = v[q];
-            }
-          }
-          // phase 2: the segment is loaded
-          __syncwarp();
-          if (lane == 0) mbar_arrive(tbar);
-          if (!mbar_wait(tbar, tphase & 1u, abort)) { aborted = true; break; }
-          ++tphase;
-          for (int kk = 0; kk < seglen; ++kk, ++kbc) {
-            const uint32_t b = kbc % NBUF;
-            if (!mbar_wait(smem_u32(&ps->tfull[b]), (kbc / NBUF) & 1u, abort)) { aborted = true; break; }
-            tc_fence_after();
-            const uint32_t taddr = tmem + (uint32_t(quad * 32) << 16) + b * NT + col0;
-            uint32_t p[CW];
-#pragma unroll
-            for (int c = 0; c + 32 <= CW; c += 32) tmem_ld32(taddr + c, *reinterpret_cast<uint32_t(*)[32]>(&p[c]));
-            if constexpr (CW % 32 == 16)
-              tmem_ld16(taddr + (CW - 16), *reinterpret_cast<uint32_t(*)[16]>(&p[CW - 16]));
-            tmem_ld_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&ps->tempty[b]));
-            const float* csk = table + kk * CW;
-#pragma unroll
-            for (int j = 0; j < CW; j += 4) {
-              const ulonglong2 sc = *reinterpret_cast<const ulonglong2*>(csk + j);
-              ffma2(acc[j / 2], p[j], p[j + 1], sc.x);
-              ffma2(acc[j / 2 + 1], p[j + 2], p[j + 3], sc.y);
-            }
-          }
+        for (int j = 0; j < CW; j += 4) {
+          const ulonglong2 sa4 = *reinterpret_cast<const ulonglong2*>(row + col0 + j);
+          ffma2(acc[j / 2], p[j], p[j + 1], fmul2(sa4.x, sw2));
+          ffma2(acc[j / 2 + 1], p[j + 2], p[j + 3], fmul2(sa4.y, sw2));
         }
-        if (aborted) break;
-        if (n_ok) {
-          const int64_t idx0 = int64_t(c0 + col0) * args.N + n;
+      }
+      if (aborted) break;
+      const int n = (cur.u % nbn) * 128 + quad * 32 + lane;   // weight row of this thread
+      if (cur.seg0 + seglen >= nkb && n < args.N) {
+        const int ncols = max(0, min(CW, min(NT, cur.r1 - cur.c0) - col0));   // valid token columns
+        const int64_t idx0 = int64_t(cur.c0 + col0) * args.N + n;
 #pragma unroll
-          for (int j = 0; j < CW; ++j) {
-            if (j < ncols) {
-              const int64_t idx = idx0 + int64_t(j) * args.N;
-              const float2 f = unpack2(acc[j / 2]);
-              const float v = (j & 1) ? f.y : f.x;
-              if (out32)
-                reinterpret_cast<float*>(args.y)[idx] = v;
-              else
-                reinterpret_cast<__nv_bfloat16*>(args.y)[idx] = __float2bfloat16_rn(v);
-            }
+        for (int j = 0; j < CW; ++j) {
+          if (j < ncols) {
+            const int64_t idx = idx0 + int64_t(j) * args.N;
+            const float2 f = unpack2(acc[j / 2]);
+            const float v = (j & 1) ? f.y : f.x;
+            if (out32)
+              reinterpret_cast<float*>(args.y)[idx] = v;
+            else
+              reinterpret_cast<__nv_bfloat16*>(args.y)[idx] = __float2bfloat16_rn(v);
           }
         }
       }
+      have = swap_seg_next<NT, KB_CAP>(args, nbn, num_units, nkb, cur);
+      ++sidx;
     }
+    cp_async_wait_all();
   }
 
   tc_fence_before();
