@@ -119,6 +119,23 @@ class ClockSampler:
                 "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
+def reduce_max(vals, dev=None):
+    """Element-wise max over all ranks of a list of floats (identity without a process
+    group).  Timings are reported as the slowest rank's."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in vals]
+    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def weak_scaling_tflops(flops_per_rank_step: float, world: int, steps: int, ms: float) -> float:
+    """Whole-job throughput: every rank runs `steps` steps of its own batch in `ms`."""
+    return flops_per_rank_step * world * steps / (ms * 1e-3) / 1e12
+
+
 def dist_setup():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -218,13 +235,10 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
 
-    if world > 1:
-        t = torch.tensor([ms, e2e_ms, aq_ms, gm_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, e2e_ms, aq_ms, gm_ms = t.tolist()
+    ms, e2e_ms, aq_ms, gm_ms = reduce_max([ms, e2e_ms, aq_ms, gm_ms], dev)
 
-    tflops = flops * world * args.steps / (ms * 1e-3) / 1e12
-    e2e_tflops = flops * world * args.steps / (e2e_ms * 1e-3) / 1e12
+    tflops = weak_scaling_tflops(flops, world, args.steps, ms)
+    e2e_tflops = weak_scaling_tflops(flops, world, args.steps, e2e_ms)
     gemm_tflops = flops / (gm_ms * 1e-3) / 1e12
     aq_bytes = M * K * 2 + M * K + M * (K // 128) * 4
     aq_gbs = aq_bytes / (aq_ms * 1e-3) / 1e9
@@ -349,22 +363,24 @@ def measure_rows(dev, peaks):
 
 def cpu_baseline_prefill(S):
     """The oracle as it stands, single-threaded, on a bounded sample of the prefill
-    workload: act_quant of 2 rows and the fp64 GEMM of 1 row x 4096 columns."""
+    workload (about 10-15 s of host time): act_quant of 3 rows and the fp64 GEMM of
+    those rows against all 28672 weight rows."""
     import oracle as O
-    K = S["K"]
-    x = S["x"][:2].cpu()
+    K, N = S["K"], S["N"]
+    rows = 3
+    x = S["x"][:rows].cpu()
     t = time.perf_counter()
     qa, sa = O.act_quant(x)
     t_aq = time.perf_counter() - t
-    qw = S["qw"][:4096].cpu().numpy()
-    sw = S["sw"][:32].cpu().numpy()
+    qw = S["qw"].cpu().numpy()
+    sw = S["sw"].cpu().numpy()
     t = time.perf_counter()
-    O.gemm_rows(qa[:1], sa[:1], qw, sw)
+    O.gemm_rows(qa, sa, qw, sw)
     t_g = time.perf_counter() - t
-    fl = 2.0 * 1 * 4096 * K
-    return {"value": round(fl / (t_aq / 2 + t_g) / 1e12, 6), "unit": "TFLOPS", "cores": 1, "kind": "oracle",
-            "sample": "act_quant of 1 row (timed on 2) + fp64 GEMM of 1 row x 4096 cols x 8192 of the "
-                      "prefill workload, single thread",
+    fl = 2.0 * rows * N * K
+    return {"value": round(fl / (t_aq + t_g) / 1e12, 6), "unit": "TFLOPS", "cores": 1, "kind": "oracle",
+            "sample": f"act_quant of {rows} rows + fp64 GEMM of {rows} rows x {N} x {K} of the prefill "
+                      "workload, single thread",
             "seconds": round(t_aq + t_g, 2)}
 
 
