@@ -125,10 +125,14 @@ int launch_act_quant(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, uint8
   constexpr int U = 2;
   const int64_t ng = (K + 127) / 128;
   const int64_t items = M * ng;
-  const int64_t per_block = (256 / 32) * 8 * U;
-  int64_t blocks = (items + per_block - 1) / per_block;
-  const int64_t cap = int64_t(num_sms()) * 8;
-  if (blocks > cap) blocks = cap;
+  // Every warp takes the same number of grid-stride steps (8 * U groups each) and
+  // the grid fits in one wave (8 resident 256-thread blocks per SM), so no warp
+  // runs a last step alone while the others idle.
+  const int64_t steps = (items + 8 * U - 1) / (8 * U);
+  const int64_t max_warps = int64_t(num_sms()) * 8 * (256 / 32);
+  const int64_t per_warp = (steps + max_warps - 1) / max_warps;
+  const int64_t warps = (steps + per_warp - 1) / per_warp;
+  const int64_t blocks = (warps + 7) / 8;
   k_act_quant<FMT, SF, U><<<int(blocks), 256, 0, st>>>(x, M, K, ldx, q, s);
   return cuda_status(cudaGetLastError());
 }

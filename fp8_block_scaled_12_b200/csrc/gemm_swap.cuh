@@ -22,7 +22,7 @@
 //   warps 4-11   promotion / epilogue: thread = one weight row (tensor-memory lane),
 //                warpgroup h = token columns [h*NT/2, (h+1)*NT/2).  Per K-block it loads
 //                all its columns in one batch, releases the buffer, then multiplies by
-//                sw * sa[token] and accumulates in fp32 registers.
+//                the table's sa[token] * sw and accumulates in fp32 registers.
 //
 // Scales.  The work of a CTA is a sequence of segments (unit, token chunk, up to
 // KB_CAP K-blocks).  A segment's scales -- sa[token][kb] for the chunk's tokens and
@@ -30,7 +30,8 @@
 // side by side so the promotion reads four columns per 16-byte load.  The epilogue
 // threads fill the table of the NEXT segment with 4-byte cp.async while they promote
 // the current one, so only the first segment's load is exposed.  The chunk's sa rows
-// are consecutive in memory, so each warp's copies read 128 contiguous bytes.
+// are consecutive in memory, so each warp's copies read 128 contiguous bytes.  Once a
+// segment has landed, its entries are multiplied by that K-block's sw in place.
 #pragma once
 
 #include "gemm.cuh"
@@ -250,7 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     SwapSeg cur;
     bool have = swap_seg_find(args, nbn, num_units, blockIdx.x, cur);
     if (have) swap_seg_load<C>(args, cur, nbn, nkb, table_s, ewarp, lane);
-    uint32_t sidx = 0, kbc = 0;
+    uint32_t sidx = 0, sph = 0, kbc = 0;
     bool aborted = false;
     uint64_t acc[CW / 2];                                // CW fp32 accumulators as packed pairs
     while (have) {
@@ -265,14 +266,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       cp_async_wait_all();
       __syncwarp();
       if (lane == 0) mbar_arrive(segbar);
-      bool ok = mbar_wait(segbar, sidx & 1u, abort);
+      bool ok = mbar_wait(segbar, sph & 1u, abort);
+      ++sph;
       if (__any_sync(0xffffffffu, !ok)) { aborted = true; break; }
       {
         SwapSeg nxt = cur;
         if (swap_seg_next<NT, KB_CAP>(args, nbn, num_units, nkb, nxt))
           swap_seg_load<C>(args, nxt, nbn, nkb, table_s + ((sidx + 1) & 1u) * C::TBUF_BYTES, ewarp, lane);
       }
-      const float* tb = table + (sidx & 1u) * (C::TBUF_BYTES / 4);
+      float* tb = table + (sidx & 1u) * (C::TBUF_BYTES / 4);
+      // Fold sw[kb] into the segment's rows once, so the promotion multiplies by one
+      // table entry per column: entry (kk, j) becomes fl32(sa * sw), the same product
+      // the promotion would form.
+      {
+        const int cnt = min(NT, cur.r1 - cur.c0);
+        for (int i = ew; i < seglen * NT; i += kEpiThreads) {
+          const int kk = i / NT, j = i - kk * NT;
+          if (j < cnt) tb[kk * C::TROW + j] = __fmul_rn(tb[kk * C::TROW + j], tb[kk * C::TROW + NT]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(segbar);
+      ok = mbar_wait(segbar, sph & 1u, abort);
+      ++sph;
+      if (__any_sync(0xffffffffu, !ok)) { aborted = true; break; }
       for (int kk = 0; kk < seglen; ++kk, ++kbc) {
         const uint32_t b = kbc % NBUF;
         ok = mbar_wait(smem_u32(&ps->tfull[b]), (kbc / NBUF) & 1u, abort);
@@ -288,14 +305,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&ps->tempty[b]));
-        const float* row = tb + kk * C::TROW;
-        const float swv = row[NT];
-        const uint64_t sw2 = pack2(swv, swv);
+        const float* row = tb + kk * C::TROW + col0;
+        // column scales in batches of 32: the loads of a batch issue back to back
 #pragma unroll
-        for (int j = 0; j < CW; j += 4) {
-          const ulonglong2 sa4 = *reinterpret_cast<const ulonglong2*>(row + col0 + j);
-          ffma2(acc[j / 2], p[j], p[j + 1], fmul2(sa4.x, sw2));
-          ffma2(acc[j / 2 + 1], p[j + 2], p[j + 3], fmul2(sa4.y, sw2));
+        for (int j0 = 0; j0 < CW; j0 += 32) {
+          constexpr int kMaxQ = 8;
+          ulonglong2 sc[kMaxQ];
+#pragma unroll
+          for (int q = 0; q < kMaxQ; ++q)
+            if (j0 + 4 * q < CW) sc[q] = *reinterpret_cast<const ulonglong2*>(row + j0 + 4 * q);
+#pragma unroll
+          for (int q = 0; q < kMaxQ; ++q)
+            if (j0 + 4 * q < CW) {
+              const int j = j0 + 4 * q;
+              ffma2(acc[j / 2], p[j], p[j + 1], sc[q].x);
+              ffma2(acc[j / 2 + 1], p[j + 2], p[j + 3], sc[q].y);
+            }
         }
       }
       if (aborted) break;
