@@ -213,27 +213,7 @@ def run_ours(args, world, rank, local):
     assert F.fp8_device_error() == 0
 
     # -------- end to end through the public API with host buffers
-    x_host = S["x"].cpu().pin_memory()
-    y_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    xd = torch.empty_like(S["x"])
-    for _ in range(max(1, args.warmup // 2)):
-        xd.copy_(x_host, non_blocking=True)
-        F.fp8_act_quant(xd, S["qa"], S["sa"], stream=stream)
-        F.fp8_block_gemm(S["qa"], S["sa"], S["qw"], S["sw"], S["y"], stream=stream)
-        y_host.copy_(S["y"], non_blocking=True)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(args.steps):
-        xd.copy_(x_host, non_blocking=True)
-        F.fp8_act_quant(xd, S["qa"], S["sa"], stream=stream)
-        F.fp8_block_gemm(S["qa"], S["sa"], S["qw"], S["sw"], S["y"], stream=stream)
-        y_host.copy_(S["y"], non_blocking=True)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
+    e2e_ms = e2e_pipelined(S, args.steps, max(1, args.warmup // 2), world)
 
     ms, e2e_ms, aq_ms, gm_ms = reduce_max([ms, e2e_ms, aq_ms, gm_ms], dev)
 
@@ -275,6 +255,59 @@ def run_ours(args, world, rank, local):
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(out), flush=True)
+
+
+def e2e_pipelined(S, steps, warm, world):
+    """Every step copies its x from pinned host memory, quantises it and multiplies
+    it (act_quant + GEMM on a compute stream) and copies y back to pinned host memory.  The
+    copies run on their own streams with two device buffers each, so step i's
+    copy-out and step i+2's copy-in overlap step i+1's kernels, as a serving loop
+    would run them.  Returns the device time from the first copy-in to the last
+    copy-out (ms)."""
+    import torch
+    import torch.distributed as dist
+    F = S["F"]
+    x_host = S["x"].cpu().pin_memory()
+    y_host = [torch.empty(S["y"].shape, dtype=S["y"].dtype).pin_memory() for _ in range(2)]
+    xd = [torch.empty_like(S["x"]) for _ in range(2)]
+    yd = [torch.empty_like(S["y"]) for _ in range(2)]
+    h2d, d2h, stream = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event(enable_timing=False)
+    x_ready, x_free, y_ready, y_free = [ev(), ev()], [ev(), ev()], [ev(), ev()], [ev(), ev()]
+
+    def run(n):
+        for b in range(2):
+            x_free[b].record(stream)
+            y_free[b].record(stream)
+        for i in range(n):
+            b = i & 1
+            h2d.wait_event(x_free[b])
+            with torch.cuda.stream(h2d):
+                xd[b].copy_(x_host, non_blocking=True)
+            x_ready[b].record(h2d)
+            stream.wait_event(x_ready[b])
+            stream.wait_event(y_free[b])
+            F.fp8_act_quant(xd[b], S["qa"], S["sa"], stream=stream)
+            x_free[b].record(stream)
+            F.fp8_block_gemm(S["qa"], S["sa"], S["qw"], S["sw"], yd[b], stream=stream)
+            y_ready[b].record(stream)
+            d2h.wait_event(y_ready[b])
+            with torch.cuda.stream(d2h):
+                y_host[b].copy_(yd[b], non_blocking=True)
+            y_free[b].record(d2h)
+
+    run(warm)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(h2d)
+    stream.wait_event(t0)
+    d2h.wait_event(t0)
+    run(steps)
+    t1.record(d2h)
+    torch.cuda.synchronize()
+    return t0.elapsed_time(t1)
 
 
 def time_launches(fn, iters, warm=2):
