@@ -246,9 +246,17 @@ __global__ void __launch_bounds__(256) k_tensor_amax(const uint16_t* __restrict_
   __shared__ float red[8];
   float a = 0.0f;
   const uint4* p = reinterpret_cast<const uint4*>(x);
-  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
-       i += int64_t(gridDim.x) * blockDim.x)
-    a = amax8(ldg_stream(p + i), a);
+  const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+  int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  // four independent 16-byte loads in flight per thread per step
+  for (; i + 3 * stride < n8; i += 4 * stride) {
+    uint4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) v[u] = ldg_stream(p + i + u * stride);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) a = amax8(v[u], a);
+  }
+  for (; i < n8; i += stride) a = amax8(ldg_stream(p + i), a);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
@@ -268,8 +276,16 @@ __global__ void __launch_bounds__(256) k_tensor_cast(const uint16_t* __restrict_
   const GroupScale<FMT, SF> sc(__uint_as_float(*amax_bits));
   const uint4* p = reinterpret_cast<const uint4*>(x);
   uint2* o = reinterpret_cast<uint2*>(q);
-  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
-       i += int64_t(gridDim.x) * blockDim.x) {
+  const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+  int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  for (; i + 3 * stride < n8; i += 4 * stride) {
+    uint4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) v[u] = ldg_stream(p + (n8 - 1 - (i + u * stride)));
+#pragma unroll
+    for (int u = 0; u < 4; ++u) o[n8 - 1 - (i + u * stride)] = quant8<FMT, SF>(v[u], sc);
+  }
+  for (; i < n8; i += stride) {
     const int64_t j = n8 - 1 - i;
     o[j] = quant8<FMT, SF>(ldg_stream(p + j), sc);
   }
