@@ -21,7 +21,7 @@ import torch
 __all__ = [
     "E4M3", "E5M2", "SCALE_FP32", "SCALE_UE8M0", "OUT_BF16", "OUT_FP32", "Fp8Error", "LIB_PATH",
     "fp8_act_quant", "fp8_weight_quant", "fp8_block_gemm", "fp8_grouped_gemm",
-    "fp8_status_string", "fp8_device_error",
+    "fp8_status_string", "fp8_device_error", "fp8_selftest_bounded_wait",
     "act_quant", "weight_quant", "block_gemm", "grouped_gemm", "EXPORTS",
 ]
 
@@ -32,7 +32,7 @@ FP8_OK = 0
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfp8lin.so")
 EXPORTS = ("fp8_act_quant", "fp8_weight_quant", "fp8_block_gemm", "fp8_grouped_gemm",
-           "fp8_status_string", "fp8_device_error")
+           "fp8_status_string", "fp8_device_error", "fp8_selftest_bounded_wait")
 
 
 class Fp8Error(RuntimeError):
@@ -43,7 +43,7 @@ class Fp8Error(RuntimeError):
 
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing; build it with `python -m fp8_block_scaled_12_b200.build`")
+        raise ImportError(f"{LIB_PATH} is missing; build it with `python fp8_block_scaled_12_b200/build.py`")
     L = ctypes.CDLL(LIB_PATH)
     vp, i64, ci = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
     L.fp8_act_quant.argtypes = [vp, i64, i64, i64, ci, ci, ci, vp, vp, vp]
@@ -53,7 +53,9 @@ def _load() -> ctypes.CDLL:
     L.fp8_status_string.argtypes = [ci]
     L.fp8_status_string.restype = ctypes.c_char_p
     L.fp8_device_error.argtypes = [vp]
-    for name in ("fp8_act_quant", "fp8_weight_quant", "fp8_block_gemm", "fp8_grouped_gemm", "fp8_device_error"):
+    L.fp8_selftest_bounded_wait.argtypes = [i64, vp]
+    for name in ("fp8_act_quant", "fp8_weight_quant", "fp8_block_gemm", "fp8_grouped_gemm", "fp8_device_error",
+                 "fp8_selftest_bounded_wait"):
         getattr(L, name).restype = ci
     return L
 
@@ -154,6 +156,12 @@ def fp8_grouped_gemm(qa: torch.Tensor, sa: torch.Tensor, qw: torch.Tensor, sw: t
 def fp8_device_error(stream=None) -> int:
     """Synchronise the stream and return (and clear) the device-side wait status."""
     return int(lib.fp8_device_error(_stream(stream)))
+
+
+def fp8_selftest_bounded_wait(limit_ns: int, stream=None) -> None:
+    """Launch the diagnostic kernel whose bounded mbarrier wait runs out after
+    `limit_ns`; a following fp8_device_error() reports the timeout."""
+    _check("fp8_selftest_bounded_wait", lib.fp8_selftest_bounded_wait(int(limit_ns), _stream(stream)))
 
 
 # ------------------------------------------------- allocating wrappers

@@ -1,6 +1,8 @@
 """Build the CUDA library libfp8lin.so in-tree with nvcc for sm_100a.
 
-    python -m fp8_block_scaled_12_b200.build [--force] [--verbose]
+    python fp8_block_scaled_12_b200/build.py [--force] [--verbose]
+
+(run by path: importing the package loads the library this script builds)
 
 The library is one translation unit (csrc/fp8lin.cu) compiled without fast-math
 (IEEE division and rounding are part of the quantisers' contract) and linked

@@ -160,6 +160,22 @@ int launch_tensor_quant(const uint16_t* x, int64_t n, uint8_t* q, float* s, cuda
   return cuda_status(cudaGetLastError());
 }
 
+// One warp whose mbarrier never completes: the bounded wait that every pipelined
+// wait of the GEMM kernels uses gives up after limit_ns, records the timeout in the
+// device error word and the kernel returns normally.
+__global__ void k_selftest_wait(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(smem_u32(&bar), 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+  if (threadIdx.x == 0) (void)mbar_wait(smem_u32(&bar), 0u, &abort_flag, limit_ns);
+  __syncwarp();
+}
+
 }  // namespace
 
 // =====================================================================
@@ -265,6 +281,12 @@ int fp8_grouped_gemm(const void* qa, const float* sa, const void* qw, const floa
   GemmArgs a{sa, sw, y, group_offsets, int(total_M), int(N), int(K), int(E),
              out_dtype == FP8_OUT_FP32 ? 1 : 0};
   return launch_swap<160, 3, 5, 28>(qa, qw, a, E * N, static_cast<cudaStream_t>(stream));
+}
+
+int fp8_selftest_bounded_wait(int64_t limit_ns, void* stream) {
+  if (limit_ns <= 0 || limit_ns > 10000000000ll) return FP8_ERR_INVALID_ARG;
+  k_selftest_wait<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(uint64_t(limit_ns));
+  return cuda_status(cudaGetLastError());
 }
 
 int fp8_device_error(void* stream) {

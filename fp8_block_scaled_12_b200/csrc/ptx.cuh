@@ -68,14 +68,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Wait until the phase with the given parity of `bar` has completed.  Returns
 // false (and raises *abort) when the wait runs out or another thread of the CTA
 // has already aborted.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
+                                          uint64_t limit_ns = FP8LIN_WAIT_NS) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1; i < FP8LIN_WAIT_ITERS; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 31u) == 0) {
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > FP8LIN_WAIT_NS) break;
+      if (globaltimer_ns() - t0 > limit_ns) break;
     }
   }
   *abort = 1;

@@ -140,6 +140,16 @@ const char* fp8_status_string(int status);
  */
 int fp8_device_error(void* stream);
 
+/*
+ * fp8_selftest_bounded_wait -- diagnostic with no counterpart in the pages.  Launches
+ * one warp on `stream` whose mbarrier is never satisfied; the same bounded wait that
+ * guards every pipelined wait of the GEMM kernels gives up after `limit_ns`
+ * nanoseconds (0 < limit_ns <= 1e10, else FP8_ERR_INVALID_ARG), sets the device-side
+ * error word and the kernel returns normally, so the CUDA context stays usable.  A
+ * following fp8_device_error() returns FP8_ERR_TIMEOUT.  Returns the launch status.
+ */
+int fp8_selftest_bounded_wait(int64_t limit_ns, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -76,6 +76,20 @@ def test_swap_path_token_counts(cuda_device, M):
     gemm_and_compare(cuda_device, M, 384, 1024, seed=M)
 
 
+@pytest.mark.parametrize("shape", [(1, 256, 8192), (64, 256, 8192), (40, 272, 7296), (100, 384, 3840), (160, 256, 3712)])
+def test_swap_path_scale_segments(cuda_device, shape):
+    """The weight-stationary kernel stages scales in segments of 56 (<= 64 tokens) or
+    28 (<= 160 tokens) K-blocks: K spans several segments with a ragged last one."""
+    M, N, K = shape
+    gemm_and_compare(cuda_device, M, N, K, seed=11 + M)
+
+
+@pytest.mark.parametrize("M", [8, 300])
+def test_single_k_block(cuda_device, M):
+    """K = 128: one K-block, one scale per row on either path."""
+    gemm_and_compare(cuda_device, M, 256, 128, seed=M)
+
+
 @pytest.mark.parametrize("shape", [(257, 512, 512), (300, 272, 640), (512, 1024, 1024), (1000, 528, 384)])
 def test_wide_path_ragged(cuda_device, shape):
     M, N, K = shape

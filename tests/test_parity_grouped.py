@@ -50,6 +50,29 @@ def test_grouped_ragged_groups(cuda_device, counts):
             check_bf16(bits_u16(y), y_ref, bound, "grouped bf16")
 
 
+def test_grouped_ragged_n_and_scale_segments(cuda_device):
+    """N = 272 (the last 128-row weight block of every expert is partial) and K spans
+    two scale segments of 28 K-blocks plus a ragged one; the last expert's tail block
+    reads past the weight tensor (zero fill) and must not disturb the others."""
+    dev = cuda_device
+    counts = [3, 170, 0, 64, 161]
+    N, K = 272, 128 * 60
+    x, w, off, (qa, sa, qw, sw) = make_grouped(dev, counts, N, K, seed=9)
+    offd = torch.from_numpy(off).to(dev)
+    T = int(off[-1])
+    rows = np.arange(0, T, 3)
+    y_ref, bound = O.grouped_gemm_rows(codes(qa), sa.cpu().numpy(), codes(qw), sw.cpu().numpy(), off, rows)
+    for out in (torch.float32, torch.bfloat16):
+        y = torch.full((T, N), float("nan"), dtype=out, device=dev)
+        F.fp8_grouped_gemm(qa, sa, qw, sw, offd, y)
+        torch.cuda.synchronize()
+        assert F.fp8_device_error() == 0
+        if out == torch.float32:
+            check_fp32(y[rows].cpu().numpy(), y_ref, bound, "grouped fp32 ragged N")
+        else:
+            check_bf16(bits_u16(y[rows]), y_ref, bound, "grouped bf16 ragged N")
+
+
 def test_grouped_leaves_rows_outside_groups_untouched(cuda_device):
     dev = cuda_device
     counts = [10, 20]
