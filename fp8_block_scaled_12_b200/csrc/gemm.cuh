@@ -68,7 +68,6 @@ struct alignas(8) PipeState {
   uint64_t empty[STAGES];
   uint64_t tfull[2];
   uint64_t tempty[2];
-  uint64_t csfull[2][2];   // swap kernel: column-scale slot handoff, [warpgroup][slot]
   uint32_t tmem_base;
   int abort;
 };

@@ -215,13 +215,6 @@ __device__ __forceinline__ void ffma2(uint64_t& acc, uint32_t p_lo, uint32_t p_h
       : "r"(p_lo), "r"(p_hi), "l"(s2));
 }
 
-// (a0*b0, a1*b1) for packed pairs, each correctly rounded (mul.rn.f32x2).
-__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-
 // ------------------------------------------------- small asynchronous copies
 // 4-byte global -> shared copy that does not block the issuing thread.
 __device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
@@ -230,10 +223,7 @@ __device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
 // Wait until every cp.async this thread issued has landed in shared memory.
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
-// --------------------------------------------------------------- misc sync
-__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
+// ------------------------------------------------------- register reallocation
 
 template <uint32_t RegCount>
 __device__ __forceinline__ void setmaxnreg_inc() {
