@@ -83,11 +83,24 @@ class ClockSampler:
             import pynvml
             pynvml.nvmlInit()
             self.nv = pynvml
-            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.h = self._handle(pynvml, index)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
             self.ok = True
         except Exception:
             self.ok = False
+
+    @staticmethod
+    def _handle(nv, index: int):
+        """NVML handle of the CUDA device `index`: NVML numbers every GPU of the host,
+        CUDA only the visible ones, so the device is matched by UUID (PCI bus id as a
+        fallback) rather than by index."""
+        import torch
+        props = torch.cuda.get_device_properties(index)
+        try:
+            return nv.nvmlDeviceGetHandleByUUID("GPU-" + str(props.uuid))
+        except Exception:
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            return nv.nvmlDeviceGetHandleByPciBusId(bus)
 
     def _run(self):
         while not self._stop.is_set():
