@@ -14,11 +14,12 @@
 // Roles (384 threads):
 //   warp 0       TMA producer: weight tile (128 rows x 128 K) plus the chunk's token
 //                rows in 32-row boxes per K-block stage.
-//   warps 1-3    MMA issuers, taking K-blocks round robin.  A thread's own barrier
-//                waits stall until the MMAs it issued before them finish, so a single
-//                issuer leaves the tensor pipe idle around every wait; with three, the
-//                others' MMAs keep it busy.  K-blocks use separate stages and buffers,
-//                so their order on the pipe does not matter.
+//   warps 1-3    MMA issuers, taking K-blocks round robin.  Issuing a K-block keeps
+//                its thread busy while the tensor pipe accepts the MMAs one by one, so
+//                a single issuer checks its barriers only between K-blocks and the
+//                pipe idles meanwhile; with three, one issuer's checks overlap the
+//                others' issue.  K-blocks use separate stages and buffers, so their
+//                order on the pipe does not matter.
 //   warps 4-11   promotion / epilogue: thread = one weight row (tensor-memory lane),
 //                warpgroup h = token columns [h*NT/2, (h+1)*NT/2).  Per K-block it loads
 //                all its columns in one batch, releases the buffer, then multiplies by
