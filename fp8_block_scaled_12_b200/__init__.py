@@ -96,6 +96,20 @@ def _u8(t: torch.Tensor) -> torch.Tensor:
     return t
 
 
+def _e4m3_codes(t: torch.Tensor, name: str) -> torch.Tensor:
+    """GEMM operands are E4M3 codes (uint8 bit patterns or float8_e4m3fn)."""
+    if t.dtype == torch.float8_e5m2:
+        raise TypeError(f"{name}: the GEMMs take E4M3 codes; float8_e5m2 is not supported")
+    return _u8(t)
+
+
+def _expect(t: torch.Tensor, shape: tuple, name: str, dtype=None) -> None:
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+
+
 # ------------------------------------------------------------- C names
 def fp8_act_quant(x: torch.Tensor, q: torch.Tensor, s: torch.Tensor, group: int = 128, fmt: int = E4M3,
                   scale_fmt: int = SCALE_FP32, stream=None) -> None:
@@ -104,6 +118,8 @@ def fp8_act_quant(x: torch.Tensor, q: torch.Tensor, s: torch.Tensor, group: int 
     assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
     assert q.is_contiguous() and s.is_contiguous() and s.dtype == torch.float32
     M, K = x.shape
+    _expect(q, (M, K), "q")
+    _expect(s, (M, (K + group - 1) // group), "s")
     _check("fp8_act_quant", lib.fp8_act_quant(_ptr(x), M, K, x.stride(0), group, fmt, scale_fmt,
                                               _ptr(_u8(q)), _ptr(s), _stream(stream)))
 
@@ -113,9 +129,15 @@ def fp8_weight_quant(w: torch.Tensor, q: torch.Tensor, s_inv: torch.Tensor, bloc
     """128x128-block (block=128) or per-tensor (block=0) quantisation of bf16 w [N, K]."""
     assert w.dtype == torch.bfloat16 and w.is_contiguous()
     assert q.is_contiguous() and s_inv.is_contiguous() and s_inv.dtype == torch.float32
-    w2 = w.reshape(-1, w.shape[-1])
-    N, K = w2.shape
-    _check("fp8_weight_quant", lib.fp8_weight_quant(_ptr(w2), N, K, block, fmt, scale_fmt, _ptr(_u8(q)),
+    if w.dim() != 2:
+        # a stacked [E, N, K] tensor would be quantised as one [E*N, K] matrix, whose
+        # 128x128 blocks straddle experts when N % 128 != 0: quantise per expert
+        raise ValueError(f"weight_quant takes one [N, K] matrix, got shape {tuple(w.shape)}; "
+                         "quantise stacked expert weights one expert at a time")
+    N, K = w.shape
+    _expect(q, (N, K), "q")
+    _expect(s_inv, (1,) if block == 0 else ((N + block - 1) // block, (K + block - 1) // block), "s_inv")
+    _check("fp8_weight_quant", lib.fp8_weight_quant(_ptr(w), N, K, block, fmt, scale_fmt, _ptr(_u8(q)),
                                                     _ptr(s_inv), _stream(stream)))
 
 
@@ -135,8 +157,13 @@ def fp8_block_gemm(qa: torch.Tensor, sa: torch.Tensor, qw: torch.Tensor, sw: tor
         assert t.is_contiguous()
     M, K = qa.shape
     N = qw.shape[0]
-    _check("fp8_block_gemm", lib.fp8_block_gemm(_ptr(_u8(qa)), _ptr(sa), _ptr(_u8(qw)), _ptr(sw), M, N, K,
-                                                _out_code(y), _ptr(y), _stream(stream)))
+    _expect(qw, (N, K), "qw")
+    _expect(sa, (M, K // 128), "sa", torch.float32)
+    _expect(sw, ((N + 127) // 128, K // 128), "sw", torch.float32)
+    _expect(y, (M, N), "y")
+    qa8, qw8, od = _e4m3_codes(qa, "qa"), _e4m3_codes(qw, "qw"), _out_code(y)
+    _check("fp8_block_gemm", lib.fp8_block_gemm(_ptr(qa8), _ptr(sa), _ptr(qw8), _ptr(sw), M, N, K,
+                                                od, _ptr(y), _stream(stream)))
 
 
 def fp8_grouped_gemm(qa: torch.Tensor, sa: torch.Tensor, qw: torch.Tensor, sw: torch.Tensor,
@@ -145,11 +172,16 @@ def fp8_grouped_gemm(qa: torch.Tensor, sa: torch.Tensor, qw: torch.Tensor, sw: t
     offsets device int32 [E+1]."""
     for t in (qa, sa, qw, sw, offsets, y):
         assert t.is_contiguous()
-    assert offsets.dtype == torch.int32
     total_M, K = qa.shape
     E, N, _ = qw.shape
-    _check("fp8_grouped_gemm", lib.fp8_grouped_gemm(_ptr(_u8(qa)), _ptr(sa), _ptr(_u8(qw)), _ptr(sw),
-                                                    _ptr(offsets), E, total_M, N, K, _out_code(y), _ptr(y),
+    _expect(qw, (E, N, K), "qw")
+    _expect(sa, (total_M, K // 128), "sa", torch.float32)
+    _expect(sw, (E, (N + 127) // 128, K // 128), "sw", torch.float32)
+    _expect(offsets, (E + 1,), "offsets", torch.int32)
+    _expect(y, (total_M, N), "y")
+    qa8, qw8, od = _e4m3_codes(qa, "qa"), _e4m3_codes(qw, "qw"), _out_code(y)
+    _check("fp8_grouped_gemm", lib.fp8_grouped_gemm(_ptr(qa8), _ptr(sa), _ptr(qw8), _ptr(sw),
+                                                    _ptr(offsets), E, total_M, N, K, od, _ptr(y),
                                                     _stream(stream)))
 
 

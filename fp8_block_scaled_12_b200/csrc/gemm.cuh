@@ -228,6 +228,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32(taddr + h * 64, p0);
           tmem_ld32(taddr + h * 64 + 32, p1);
           tmem_ld_wait();
+          tmem_regs_ready(p0);
+          tmem_regs_ready(p1);
           if (h == 1) {
             tc_fence_before();
             __syncwarp();

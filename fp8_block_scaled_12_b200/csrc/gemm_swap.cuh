@@ -80,10 +80,12 @@ __device__ __forceinline__ void group_range(const GemmArgs& a, int e, int& r0, i
     r0 = 0;
     r1 = a.M;
   } else {
+    // clamp into [0, M] so a malformed offsets table can only shrink the work,
+    // never address rows outside qa / sa / y
     r0 = __ldg(a.offsets + e);
     r1 = __ldg(a.offsets + e + 1);
-    r1 = min(r1, a.M);
-    r0 = min(r0, r1);
+    r1 = min(max(r1, 0), a.M);
+    r0 = min(max(r0, 0), r1);
   }
 }
 
@@ -303,6 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if constexpr (CW % 32 == 16)
           tmem_ld16(taddr + (CW - 16), *reinterpret_cast<uint32_t(*)[16]>(&p[CW - 16]));
         tmem_ld_wait();
+        tmem_regs_ready(p);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&ps->tempty[b]));

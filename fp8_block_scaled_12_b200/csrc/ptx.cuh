@@ -177,6 +177,17 @@ __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// Call right after tmem_ld_wait() on every register array it completed.  The
+// registers pass through an empty volatile asm that the compiler keeps after the
+// (volatile) wait, so every later use of them -- including non-volatile
+// arithmetic asm such as ffma2 -- depends on the wait and cannot be hoisted above
+// it.  Emits no instruction.
+template <int N>
+__device__ __forceinline__ void tmem_regs_ready(uint32_t (&r)[N]) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
+}
+
 // Shared-memory matrix descriptor for a K-major operand tile written by TMA with
 // the 128-byte swizzle: rows of 128 bytes, 8-row atoms of 1024 bytes stacked
 // contiguously (stride 1024 B between atoms).  Fields: start address >> 4 in

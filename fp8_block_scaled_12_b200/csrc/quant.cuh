@@ -51,10 +51,13 @@ __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w 
 // IEEE division per element.  Groups
 // with s < 2^-64 first scale x and s by 2^64 (exact) so every residual that can
 // decide a code stays a normal number.  For every bf16 amax and every bf16 x with
-// |x| <= amax this gives the same FP8 code as fl32(x / s) rounded to nearest even
-// (checked exhaustively, E4M3 and E5M2: tests/test_division_identity.py); the fp32
-// quotients themselves may differ only where they are far below the smallest FP8
-// subnormal.
+// |x| <= amax this gives the same FP8 code as fl32(x / s) rounded to nearest even:
+// tests/division_identity.c restates this arithmetic on the host and compares codes.
+// Its exhaustive run (every bf16 amax, 2 x 1,065,402,238 (amax, x) pairs, E4M3 and
+// E5M2, 0 mismatches) is recorded in tests/golden/division_identity_exhaustive.txt;
+// tests/test_division_identity.py reruns it stratified by default and exhaustively
+// with FP8LIN_EXHAUSTIVE=1.  The fp32 quotients themselves may differ only where
+// they are far below the smallest FP8 subnormal.
 // ue8m0 scales: a multiplication by the exact power of two 2^-e, which rounds
 // identically to the IEEE quotient (same exact value, one rounding).
 template <int FMT, int SF>

@@ -13,6 +13,7 @@ from __future__ import annotations
 
 import ctypes
 import os
+from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
 
@@ -57,6 +58,31 @@ def lib():
         del u8p
         _lib = L
     return _lib
+
+
+def default_threads() -> int:
+    """Host threads the row-parallel helpers use: every core this process may run on."""
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:
+        return max(1, os.cpu_count() or 1)
+
+
+def _split(n: int, parts: int, align: int = 1):
+    """[start, stop) ranges covering [0, n) in at most `parts` pieces, boundaries on multiples of align."""
+    units = (n + align - 1) // align
+    parts = max(1, min(parts, units))
+    bounds = [min(n, (units * i // parts) * align) for i in range(parts + 1)]
+    return [(a, b) for a, b in zip(bounds[:-1], bounds[1:]) if b > a]
+
+
+def _run_parallel(fn, ranges, threads: int):
+    """Run fn(start, stop) over the ranges on `threads` host threads (the C calls
+    release the GIL), in order of the ranges."""
+    if threads <= 1 or len(ranges) <= 1:
+        return [fn(a, b) for a, b in ranges]
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        return list(ex.map(lambda r: fn(*r), ranges))
 
 
 def _ptr(a: np.ndarray) -> int:
@@ -105,19 +131,26 @@ def round_bf16(v: np.ndarray) -> np.ndarray:
 
 
 # ------------------------------------------------------------ quantisers
-def act_quant(x, group: int = 128, fmt: int = E4M3, scale_fmt: int = SCALE_FP32):
-    """x: [M, K] bf16 (bits or torch tensor) -> (q uint8 [M, K], s fp32 [M, ceil(K/group)])."""
+def act_quant(x, group: int = 128, fmt: int = E4M3, scale_fmt: int = SCALE_FP32, threads: int = 1):
+    """x: [M, K] bf16 (bits or torch tensor) -> (q uint8 [M, K], s fp32 [M, ceil(K/group)]).
+    threads > 1 splits the rows (independent) over host threads."""
     xb = _bf16_bits(x)
     M, K = xb.shape
     ng = (K + group - 1) // group
     q = np.empty((M, K), dtype=np.uint8)
     s = np.empty((M, ng), dtype=np.float32)
-    lib().orc_act_quant(_ptr(xb), M, K, K, group, fmt, scale_fmt, _ptr(q), _ptr(s))
+
+    def part(r0, r1):
+        lib().orc_act_quant(_ptr(xb) + r0 * K * 2, r1 - r0, K, K, group, fmt, scale_fmt,
+                            _ptr(q) + r0 * K, _ptr(s) + r0 * ng * 4)
+
+    _run_parallel(part, _split(M, threads), threads)
     return q, s
 
 
-def weight_quant(w, block: int = 128, fmt: int = E4M3, scale_fmt: int = SCALE_FP32):
-    """w: [N, K] bf16 -> (q uint8 [N, K], s_inv fp32 [ceil(N/b), ceil(K/b)]); block=0 is per-tensor."""
+def weight_quant(w, block: int = 128, fmt: int = E4M3, scale_fmt: int = SCALE_FP32, threads: int = 1):
+    """w: [N, K] bf16 -> (q uint8 [N, K], s_inv fp32 [ceil(N/b), ceil(K/b)]); block=0 is per-tensor.
+    threads > 1 splits the block rows (independent) over host threads."""
     wb = _bf16_bits(w)
     N, K = wb.shape
     q = np.empty((N, K), dtype=np.uint8)
@@ -125,8 +158,14 @@ def weight_quant(w, block: int = 128, fmt: int = E4M3, scale_fmt: int = SCALE_FP
         s = np.empty((1,), dtype=np.float32)
         lib().orc_tensor_quant(_ptr(wb), N * K, fmt, scale_fmt, _ptr(q), _ptr(s))
         return q, s
-    s = np.empty(((N + block - 1) // block, (K + block - 1) // block), dtype=np.float32)
-    lib().orc_weight_quant_block(_ptr(wb), N, K, block, fmt, scale_fmt, _ptr(q), _ptr(s))
+    nbk = (K + block - 1) // block
+    s = np.empty(((N + block - 1) // block, nbk), dtype=np.float32)
+
+    def part(r0, r1):
+        lib().orc_weight_quant_block(_ptr(wb) + r0 * K * 2, r1 - r0, K, block, fmt, scale_fmt,
+                                     _ptr(q) + r0 * K, _ptr(s) + (r0 // block) * nbk * 4)
+
+    _run_parallel(part, _split(N, threads, block), threads)
     return q, s
 
 
@@ -148,8 +187,9 @@ def cast_with_scale(x, s: float, fmt: int = E4M3):
 
 
 # ------------------------------------------------------------------ GEMM
-def gemm_rows(qa, sa, qw, sw, rows=None):
-    """fp64 block-scaled GEMM on the given rows -> (y [nr, N] fp64, bound [nr, N] fp64)."""
+def gemm_rows(qa, sa, qw, sw, rows=None, threads: int = 1):
+    """fp64 block-scaled GEMM on the given rows -> (y [nr, N] fp64, bound [nr, N] fp64).
+    threads > 1 splits the rows over host threads."""
     qa = np.ascontiguousarray(qa, dtype=np.uint8)
     qw = np.ascontiguousarray(qw, dtype=np.uint8)
     sa = np.ascontiguousarray(sa, dtype=np.float32)
@@ -160,12 +200,18 @@ def gemm_rows(qa, sa, qw, sw, rows=None):
     rows = np.arange(M, dtype=np.int64) if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
     y = np.empty((rows.size, N), dtype=np.float64)
     b = np.empty((rows.size, N), dtype=np.float64)
-    lib().orc_gemm_rows(_ptr(qa), _ptr(sa), _ptr(qw), _ptr(sw), N, K, _ptr(rows), rows.size, _ptr(y), _ptr(b))
+
+    def part(i0, i1):
+        lib().orc_gemm_rows(_ptr(qa), _ptr(sa), _ptr(qw), _ptr(sw), N, K, _ptr(rows) + i0 * 8, i1 - i0,
+                            _ptr(y) + i0 * N * 8, _ptr(b) + i0 * N * 8)
+
+    _run_parallel(part, _split(rows.size, threads), threads)
     return y, b
 
 
-def grouped_gemm_rows(qa, sa, qw, sw, offsets, rows):
-    """Grouped GEMM on selected rows.  qw: [E, N, K], sw: [E, ceil(N/128), K/128], offsets int32 [E+1]."""
+def grouped_gemm_rows(qa, sa, qw, sw, offsets, rows, threads: int = 1):
+    """Grouped GEMM on selected rows.  qw: [E, N, K], sw: [E, ceil(N/128), K/128], offsets int32 [E+1].
+    threads > 1 splits the rows over host threads."""
     qa = np.ascontiguousarray(qa, dtype=np.uint8)
     qw = np.ascontiguousarray(qw, dtype=np.uint8)
     sa = np.ascontiguousarray(sa, dtype=np.float32)
@@ -175,6 +221,10 @@ def grouped_gemm_rows(qa, sa, qw, sw, offsets, rows):
     rows = np.ascontiguousarray(rows, dtype=np.int64)
     y = np.empty((rows.size, N), dtype=np.float64)
     b = np.empty((rows.size, N), dtype=np.float64)
-    lib().orc_grouped_gemm_rows(_ptr(qa), _ptr(sa), _ptr(qw), _ptr(sw), _ptr(off), E, N, K,
-                                _ptr(rows), rows.size, _ptr(y), _ptr(b))
+
+    def part(i0, i1):
+        lib().orc_grouped_gemm_rows(_ptr(qa), _ptr(sa), _ptr(qw), _ptr(sw), _ptr(off), E, N, K,
+                                    _ptr(rows) + i0 * 8, i1 - i0, _ptr(y) + i0 * N * 8, _ptr(b) + i0 * N * 8)
+
+    _run_parallel(part, _split(rows.size, threads), threads)
     return y, b

@@ -23,7 +23,8 @@
  *  [P5] "量化：FP8 与混合精度推理" (charles2530.github.io), "FP8 也需要 scale":
  *       x_fp8 = FP8Cast(x / s), x_hat = s * x_fp8.
  *
- * Readings taken where the pages are silent (each one is listed in the design doc):
+ * Readings taken where the pages are silent or disagree (scale direction: [P3]
+ * and [P5] divide where [P2] multiplies; the rest is not stated on any page):
  *  - the scale divides (x / s), it is stored as the dequantisation multiplier;
  *  - the division x / s is one IEEE fp32 division, then round-to-nearest-even
  *    to FP8 with saturation to +-Fmax (no Inf is ever produced);
@@ -231,19 +232,33 @@ void orc_tensor_quant(const uint16_t *x, int64_t n, int fmt, int scale_fmt,
  *   y[m][n] = sum_k (dec(qa[m][k]) * sa[m][k/128]) * (dec(qw[n][k]) * sw[n/128][k/128])
  * summed in fp64 in k order.  bound[m][n] = sum_k |a_k * w_k| (the tolerance
  * scale).  rows lists the nr rows to compute; outputs are [nr][N]. */
+/* Decoded value of every E4M3 code, filled once by orc_decode so the GEMM's inner
+ * loop looks values up instead of re-deriving them (same doubles, fewer calls). */
+static double g_dec_e4m3[256];
+static int g_dec_ready;
+
+static const double *e4m3_values(void)
+{
+    if (!g_dec_ready) {
+        for (int c = 0; c < 256; ++c) g_dec_e4m3[c] = orc_decode((uint8_t)c, ORC_E4M3);
+        g_dec_ready = 1;
+    }
+    return g_dec_e4m3;
+}
+
 void orc_gemm_rows(const uint8_t *qa, const float *sa, const uint8_t *qw, const float *sw,
                    int64_t N, int64_t K, const int64_t *rows, int64_t nr,
                    double *y, double *bound)
 {
     const int64_t nkb = K / 128;
+    const double *dec = e4m3_values();
     for (int64_t i = 0; i < nr; ++i) {
         int64_t m = rows[i];
         for (int64_t n = 0; n < N; ++n) {
             double acc = 0.0, b = 0.0;
             for (int64_t k = 0; k < K; ++k) {
-                double a = orc_decode(qa[m * K + k], ORC_E4M3) * (double)sa[m * nkb + k / 128];
-                double w = orc_decode(qw[n * K + k], ORC_E4M3) *
-                           (double)sw[(n / 128) * nkb + k / 128];
+                double a = dec[qa[m * K + k]] * (double)sa[m * nkb + k / 128];
+                double w = dec[qw[n * K + k]] * (double)sw[(n / 128) * nkb + k / 128];
                 acc += a * w;
                 b += fabs(a * w);
             }

@@ -91,3 +91,46 @@ def test_python_binding_rejects_host_tensors():
     x = torch.zeros(4, 128, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         F.fp8_act_quant(x, torch.zeros(4, 128, dtype=torch.uint8), torch.zeros(4, 1))
+
+
+def test_python_binding_checks_gemm_operands():
+    """The GEMM wrappers refuse E5M2 codes (the kernels decode E4M3) and operands
+    whose shapes disagree with qa / qw, before anything reaches the library."""
+    import torch
+    M, N, K = 4, 256, 256
+    qa = torch.zeros(M, K, dtype=torch.uint8)
+    sa = torch.zeros(M, K // 128)
+    qw = torch.zeros(N, K, dtype=torch.uint8)
+    sw = torch.zeros(N // 128, K // 128)
+    y = torch.zeros(M, N, dtype=torch.bfloat16)
+    with pytest.raises(TypeError):
+        F.fp8_block_gemm(qa.view(torch.float8_e5m2), sa, qw, sw, y)
+    with pytest.raises(TypeError):
+        F.fp8_block_gemm(qa, sa, qw.view(torch.float8_e5m2), sw, y)
+    with pytest.raises(ValueError):
+        F.fp8_block_gemm(qa, sa, torch.zeros(N, K + 128, dtype=torch.uint8), sw, y)   # K differs
+    with pytest.raises(ValueError):
+        F.fp8_block_gemm(qa, torch.zeros(M, K // 128 + 1), qw, sw, y)                 # sa shape
+    with pytest.raises(ValueError):
+        F.fp8_block_gemm(qa, sa, qw, torch.zeros(1, K // 128), y)                     # sw shape
+    with pytest.raises(ValueError):
+        F.fp8_block_gemm(qa, sa, qw, sw, torch.zeros(M, N + 16, dtype=torch.bfloat16))
+    E = 3
+    qwe = torch.zeros(E, N, K, dtype=torch.uint8)
+    swe = torch.zeros(E, N // 128, K // 128)
+    off = torch.zeros(E + 1, dtype=torch.int32)
+    with pytest.raises(ValueError):
+        F.fp8_grouped_gemm(qa, sa, qwe, swe, torch.zeros(E, dtype=torch.int32), y)    # offsets [E+1]
+    with pytest.raises(TypeError):
+        F.fp8_grouped_gemm(qa, sa, qwe, swe, off.to(torch.int64), y)
+    with pytest.raises(ValueError):
+        F.fp8_grouped_gemm(qa, sa, qwe, swe[:, :1].contiguous(), off, y)
+
+
+def test_python_binding_refuses_stacked_weights():
+    """A stacked [E, N, K] weight would be quantised as one [E*N, K] matrix whose
+    128x128 blocks straddle experts; the wrapper refuses it."""
+    import torch
+    w = torch.zeros(2, 200, 256, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        F.fp8_weight_quant(w, torch.zeros(2, 200, 256, dtype=torch.uint8), torch.zeros(4, 2))

@@ -14,7 +14,7 @@ import torch
 import fp8_block_scaled_12_b200 as F
 import oracle as O
 import synth
-from _parity import assert_codes_equal, assert_scales_equal, bits_u16, check_bf16, check_fp32, codes
+from _parity import THREADS, assert_codes_equal, assert_scales_equal, bits_u16, check_bf16, check_fp32, codes
 
 pytestmark = pytest.mark.gpu
 
@@ -34,10 +34,10 @@ def quantise_both(x, w, sf, dev):
 def oracle_check_quant(x, w, sf, h, rows=None):
     osf = O.SCALE_FP32 if sf == F.SCALE_FP32 else O.SCALE_UE8M0
     xs = x if rows is None else x[rows]
-    qar, sar = O.act_quant(xs, scale_fmt=osf)
+    qar, sar = O.act_quant(xs, scale_fmt=osf, threads=THREADS)
     assert_codes_equal(h["qa"] if rows is None else h["qa"][rows], qar, "activation codes")
     assert_scales_equal(h["sa"] if rows is None else h["sa"][rows], sar, "activation scales")
-    qwr, swr = O.weight_quant(w, scale_fmt=osf)
+    qwr, swr = O.weight_quant(w, scale_fmt=osf, threads=THREADS)
     assert_codes_equal(h["qw"], qwr, "weight codes")
     assert_scales_equal(h["sw"], swr, "weight scales")
 
@@ -49,7 +49,7 @@ def gemm_and_compare(dev, M, N, K, sf=F.SCALE_FP32, rows=None, outs=("bf16", "fp
     (qa, sa, qw, sw), h = quantise_both(x, w, sf, dev)
     if check_weights:
         oracle_check_quant(x, w, sf, h, rows)
-    y_ref, bound = O.gemm_rows(h["qa"], h["sa"], h["qw"], h["sw"], rows=rows)
+    y_ref, bound = O.gemm_rows(h["qa"], h["sa"], h["qw"], h["sw"], rows=rows, threads=THREADS)
     sel = slice(None) if rows is None else torch.as_tensor(rows, device=dev)
     allowed = 0
     for o in outs:
@@ -154,9 +154,36 @@ def test_prefill_config_full_size(cuda_device):
     qar, sar = O.act_quant(x[rows].cpu())
     assert_codes_equal(hq["qa"], qar, "activation codes")
     assert_scales_equal(hq["sa"], sar, "activation scales")
-    # weight codes for the first 256 rows (two row-blocks) against the oracle
-    qwr, swr = O.weight_quant(w[:256].cpu())
-    assert_codes_equal(hq["qw"][:256], qwr, "weight codes (first 256 rows)")
-    assert_scales_equal(hq["sw"][:2], swr, "weight scales (first 2 row-blocks)")
-    y_ref, bound = O.gemm_rows(hq["qa"], hq["sa"], hq["qw"], hq["sw"])
+    # every weight code and block scale against the oracle (row blocks split over host threads)
+    qwr, swr = O.weight_quant(w.cpu(), threads=THREADS)
+    assert_codes_equal(hq["qw"], qwr, "weight codes (all 28672 rows)")
+    assert_scales_equal(hq["sw"], swr, "weight scales (all 224 x 64 blocks)")
+    del qwr
+    y_ref, bound = O.gemm_rows(hq["qa"], hq["sa"], hq["qw"], hq["sw"], threads=THREADS)
     check_bf16(bits_u16(y[rows]), y_ref, bound, "prefill bf16")
+
+
+# --------------------------------------------------------------------------
+# Persistent loops: sizes at which every CTA of the (SM-count sized) grid runs
+# at least three work items, compared element by element.
+
+
+def test_wide_persistent_multi_tile(cuda_device):
+    """M=2048, N=7168: 16 x 28 = 448 tiles of 128 x 256 over at most 148 CTAs (>= 3 tiles
+    each).  K = 384 is three K-blocks, an odd count, so the tensor-memory buffer and its
+    phase alternate differently from one tile to the next.  Every element, fp32 and bf16."""
+    gemm_and_compare(cuda_device, 2048, 7168, 384, seed=21)
+
+
+@pytest.mark.parametrize("M", [40, 150])
+def test_swap_dense_multi_unit(cuda_device, M):
+    """Few-token path with N = 57344: 448 units of 128 weight rows over at most 148 CTAs
+    (>= 3 units each), for both token tiles (M <= 64 and 64 < M <= 160).  Every element."""
+    gemm_and_compare(cuda_device, M, 57344, 384, seed=M + 3)
+
+
+def test_swap_dense_multi_unit_multi_segment(cuda_device):
+    """M = 65 (token tile 160, 28 K-blocks per scale segment) and K = 29 K-blocks: each
+    of the >= 3 units per CTA has a full and a one-K-block segment, so the two
+    scale-table buffers alternate inside and across units.  Every element."""
+    gemm_and_compare(cuda_device, 65, 56832, 29 * 128, seed=29, outs=("bf16",))

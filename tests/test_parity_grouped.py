@@ -6,7 +6,7 @@ import torch
 import fp8_block_scaled_12_b200 as F
 import oracle as O
 import synth
-from _parity import assert_codes_equal, assert_scales_equal, bits_u16, check_bf16, check_fp32, codes
+from _parity import THREADS, assert_codes_equal, assert_scales_equal, bits_u16, check_bf16, check_fp32, codes
 
 pytestmark = pytest.mark.gpu
 
@@ -38,7 +38,8 @@ def test_grouped_ragged_groups(cuda_device, counts):
     offd = torch.from_numpy(off).to(dev)
     T = int(off[-1])
     rows = np.arange(T)
-    y_ref, bound = O.grouped_gemm_rows(codes(qa), sa.cpu().numpy(), codes(qw), sw.cpu().numpy(), off, rows)
+    y_ref, bound = O.grouped_gemm_rows(codes(qa), sa.cpu().numpy(), codes(qw), sw.cpu().numpy(), off, rows,
+                                       threads=THREADS)
     for out in (torch.float32, torch.bfloat16):
         y = torch.full((T, N), float("nan"), dtype=out, device=dev)
         F.fp8_grouped_gemm(qa, sa, qw, sw, offd, y)
@@ -61,7 +62,8 @@ def test_grouped_ragged_n_and_scale_segments(cuda_device):
     offd = torch.from_numpy(off).to(dev)
     T = int(off[-1])
     rows = np.arange(0, T, 3)
-    y_ref, bound = O.grouped_gemm_rows(codes(qa), sa.cpu().numpy(), codes(qw), sw.cpu().numpy(), off, rows)
+    y_ref, bound = O.grouped_gemm_rows(codes(qa), sa.cpu().numpy(), codes(qw), sw.cpu().numpy(), off, rows,
+                                       threads=THREADS)
     for out in (torch.float32, torch.bfloat16):
         y = torch.full((T, N), float("nan"), dtype=out, device=dev)
         F.fp8_grouped_gemm(qa, sa, qw, sw, offd, y)
@@ -111,18 +113,19 @@ def test_moe_config_full_size(cuda_device):
     qw = torch.empty((E, N, K), dtype=torch.uint8, device=dev)
     sw = torch.empty((E, N // 128, K // 128), dtype=torch.float32, device=dev)
     experts = [0, 1, 17, 64, 100, 128, 150, 200, 201, 230, 254, 255]
+    checked = experts[::2]                       # weight codes of 6 experts (88 M codes)
     w_keep = {}
     for e in range(E):
         we = synth.weights(N, K, p["w_std"], seed=0, chunk=e, device=dev)
         F.fp8_weight_quant(we, qw[e], sw[e])
-        if e in experts[:2]:
+        if e in checked:
             w_keep[e] = we.cpu()
     offd = off.to(dev)
     y = F.grouped_gemm(qa, sa, qw, sw, offd)
     torch.cuda.synchronize()
     assert F.fp8_device_error() == 0
-    for e in experts[:2]:
-        qwr, swr = O.weight_quant(w_keep[e])
+    for e in checked:
+        qwr, swr = O.weight_quant(w_keep[e], threads=THREADS)
         assert_codes_equal(codes(qw[e]), qwr, f"expert {e} weight codes")
         assert_scales_equal(sw[e].cpu().numpy(), swr, f"expert {e} weight scales")
     offn = off.numpy()
@@ -135,3 +138,49 @@ def test_moe_config_full_size(cuda_device):
         assert_codes_equal(codes(qa[rows]), qar, "activation codes")
         y_ref, bound = O.gemm_rows(codes(qa[rows]), sa[rows].cpu().numpy(), codes(qw[e]), sw[e].cpu().numpy())
         check_bf16(bits_u16(y[rows]), y_ref, bound, f"moe expert {e}")
+
+
+def _grouped_full_compare(dev, counts, N, K, seed, outs=(torch.float32, torch.bfloat16)):
+    x, w, off, (qa, sa, qw, sw) = make_grouped(dev, counts, N, K, seed=seed)
+    qar, sar = O.act_quant(x, threads=THREADS)
+    assert_codes_equal(codes(qa), qar, "activation codes")
+    assert_scales_equal(sa.cpu().numpy(), sar, "activation scales")
+    offd = torch.from_numpy(off).to(dev)
+    T = int(off[-1])
+    rows = np.arange(T)
+    y_ref, bound = O.grouped_gemm_rows(codes(qa), sa.cpu().numpy(), codes(qw), sw.cpu().numpy(), off, rows,
+                                       threads=THREADS)
+    for out in outs:
+        y = torch.full((T, N), float("nan"), dtype=out, device=dev)
+        F.fp8_grouped_gemm(qa, sa, qw, sw, offd, y)
+        torch.cuda.synchronize()
+        assert F.fp8_device_error() == 0
+        if out == torch.float32:
+            check_fp32(y.cpu().numpy(), y_ref, bound, f"grouped fp32 E={len(counts)} N={N} K={K}")
+        else:
+            check_bf16(bits_u16(y), y_ref, bound, f"grouped bf16 E={len(counts)} N={N} K={K}")
+
+
+def _ragged_counts(E, seed, hi=90):
+    """Seeded ragged expert sizes with empty experts, single-row experts and experts
+    larger than one 160-token chunk."""
+    rng = np.random.default_rng(seed)
+    c = rng.integers(0, hi, E)
+    c[rng.choice(E, E // 8, replace=False)] = 0
+    c[rng.choice(E, 3, replace=False)] = 1
+    c[rng.choice(E, 2, replace=False)] = 170
+    return c.tolist()
+
+
+def test_grouped_persistent_multi_unit(cuda_device):
+    """E = 64 experts x N = 1024 (8 weight blocks each): 512 units over at most 148 CTAs
+    (>= 3 each), ragged and empty experts.  Every element, fp32 and bf16."""
+    _grouped_full_compare(cuda_device, _ragged_counts(64, 5), 1024, 512, seed=31)
+
+
+def test_grouped_persistent_multi_unit_multi_segment(cuda_device):
+    """Same unit count with K = 29 K-blocks: each unit has a 28-K-block and a 1-K-block
+    scale segment, so the scale tables alternate inside units, across units and across
+    experts.  Every element."""
+    _grouped_full_compare(cuda_device, _ragged_counts(64, 6, hi=30), 1024, 29 * 128, seed=32,
+                          outs=(torch.bfloat16,))

@@ -8,7 +8,7 @@ import torch
 import fp8_block_scaled_12_b200 as F
 import oracle as O
 import synth
-from _parity import assert_codes_equal, assert_scales_equal, codes
+from _parity import THREADS, assert_codes_equal, assert_scales_equal, codes
 
 pytestmark = pytest.mark.gpu
 
@@ -99,7 +99,7 @@ def test_act_quant_sweep_sizes(cuda_device, sf):
     for M in (1024, 4096):
         x = synth.activations(M, K, seed=0, dist="t3", device=cuda_device)
         q, s = F.act_quant(x, scale_fmt=sf[0])
-        qr, sr = O.act_quant(x.cpu(), scale_fmt=sf[1])
+        qr, sr = O.act_quant(x.cpu(), scale_fmt=sf[1], threads=THREADS)
         assert_codes_equal(codes(q), qr, f"codes M={M}")
         assert_scales_equal(s.cpu().numpy(), sr, f"scales M={M}")
     x = synth.activations(16384, K, seed=0, dist="t3", device=cuda_device)
@@ -111,33 +111,37 @@ def test_act_quant_sweep_sizes(cuda_device, sf):
     assert_scales_equal(s[rows.to(cuda_device)].cpu().numpy(), sr, "scales M=16384 (sampled rows)")
 
 
+@pytest.mark.parametrize("fmt", FMTS, ids=["e4m3", "e5m2"])
 @pytest.mark.parametrize("sf", SFS, ids=["fp32", "ue8m0"])
 @pytest.mark.parametrize("shape", [(256, 512), (300, 272), (18432 // 8, 7168)])
-def test_weight_block_quant(cuda_device, sf, shape):
+def test_weight_block_quant(cuda_device, fmt, sf, shape):
+    """128 x 128 blocks, E4M3 and E5M2 codes, fp32 and ue8m0 scales; ragged edge blocks;
+    one block carries an outlier.  Every code and scale."""
     N, K = shape
     w = synth.weights(N, K, 0.02, seed=1, device=cuda_device)
     w[min(N - 1, 130), min(K - 1, 260)] = 3.0      # one block with an outlier
-    q, s = F.weight_quant(w, block=128, scale_fmt=sf[0])
-    qr, sr = O.weight_quant(w.cpu(), block=128, scale_fmt=sf[1])
+    q, s = F.weight_quant(w, block=128, fmt=fmt[0], scale_fmt=sf[0])
+    qr, sr = O.weight_quant(w.cpu(), block=128, fmt=fmt[1], scale_fmt=sf[1], threads=THREADS)
     assert_codes_equal(codes(q), qr, "codes")
     assert_scales_equal(s.cpu().numpy(), sr, "scales")
 
 
 @pytest.mark.parametrize("fmt", FMTS, ids=["e4m3", "e5m2"])
+@pytest.mark.parametrize("sf", SFS, ids=["fp32", "ue8m0"])
 @pytest.mark.parametrize("shape", [(64, 256), (1024, 7168), (16384, 7168)])
-def test_per_tensor_quant(cuda_device, fmt, shape):
+def test_per_tensor_quant(cuda_device, fmt, sf, shape):
     M, K = shape
     x = synth.activations(M, K, seed=2, dist="t3", device=cuda_device)
-    q, s = F.weight_quant(x, block=0, fmt=fmt[0])
+    q, s = F.weight_quant(x, block=0, fmt=fmt[0], scale_fmt=sf[0])
     torch.cuda.synchronize()
     if M * K <= 8_000_000:
-        qr, sr = O.tensor_quant(x.cpu(), fmt=fmt[1])
+        qr, sr = O.tensor_quant(x.cpu(), fmt=fmt[1], scale_fmt=sf[1])
         assert_codes_equal(codes(q), qr, "codes")
     else:
         # the scale depends on every element: take the amax on the host (exact), then
         # check the oracle's cast under that scale on a row sample
         amax = float(x.abs().max().float())
-        sr = np.array([O.scale_from_amax(amax, fmt[1], O.SCALE_FP32)], np.float32)
+        sr = np.array([O.scale_from_amax(amax, fmt[1], sf[1])], np.float32)
         rows = torch.arange(0, M, 97, device=cuda_device)
         qr = O.cast_with_scale(x[rows].cpu(), float(sr[0]), fmt[1])
         assert_codes_equal(codes(q[rows]), qr, "codes (sampled rows)")
