@@ -53,6 +53,12 @@ def lib():
         L.orc_tensor_quant.argtypes = [vp, i64, ctypes.c_int, ctypes.c_int, vp, vp]
         L.orc_gemm_rows.restype = None
         L.orc_gemm_rows.argtypes = [vp, vp, vp, vp, i64, i64, vp, i64, vp, vp]
+        L.orc_e8m0_decode.restype = ctypes.c_double
+        L.orc_e8m0_decode.argtypes = [ctypes.c_uint8]
+        L.orc_mx_quant.restype = None
+        L.orc_mx_quant.argtypes = [vp, i64, i64, i64, i64, ctypes.c_int, vp, vp]
+        L.orc_mx_gemm_rows.restype = None
+        L.orc_mx_gemm_rows.argtypes = [vp, vp, vp, vp, i64, i64, vp, i64, vp, vp]
         L.orc_grouped_gemm_rows.restype = None
         L.orc_grouped_gemm_rows.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp, i64, vp, vp]
         del u8p
@@ -225,6 +231,55 @@ def grouped_gemm_rows(qa, sa, qw, sw, offsets, rows, threads: int = 1):
     def part(i0, i1):
         lib().orc_grouped_gemm_rows(_ptr(qa), _ptr(sa), _ptr(qw), _ptr(sw), _ptr(off), E, N, K,
                                     _ptr(rows) + i0 * 8, i1 - i0, _ptr(y) + i0 * N * 8, _ptr(b) + i0 * N * 8)
+
+    _run_parallel(part, _split(rows.size, threads), threads)
+    return y, b
+
+
+# ----------------------------------------------------------------- MXFP8
+MX_BLOCK = 32
+
+
+def e8m0_decode(b: int) -> float:
+    """Value 2^(b-127) of an E8M0 shared-exponent byte (0xFF is NaN)."""
+    return lib().orc_e8m0_decode(b & 0xFF)
+
+
+def mx_quant(x, fmt: int = E4M3, block: int = MX_BLOCK, threads: int = 1):
+    """MXFP8: x [M, K] bf16 -> (q uint8 [M, K], e8 uint8 [M, ceil(K/block)]) with one E8M0
+    exponent per `block` consecutive elements of a row."""
+    xb = _bf16_bits(x)
+    M, K = xb.shape
+    nb = (K + block - 1) // block
+    q = np.empty((M, K), dtype=np.uint8)
+    e8 = np.empty((M, nb), dtype=np.uint8)
+
+    def part(r0, r1):
+        lib().orc_mx_quant(_ptr(xb) + r0 * K * 2, r1 - r0, K, K, block, fmt, _ptr(q) + r0 * K,
+                           _ptr(e8) + r0 * nb)
+
+    _run_parallel(part, _split(M, threads), threads)
+    return q, e8
+
+
+def mx_gemm_rows(qa, ea, qw, ew, rows=None, threads: int = 1):
+    """fp64 MXFP8 GEMM on the given rows (32-element E8M0 blocks along K on both
+    operands) -> (y [nr, N], bound [nr, N])."""
+    qa = np.ascontiguousarray(qa, dtype=np.uint8)
+    qw = np.ascontiguousarray(qw, dtype=np.uint8)
+    ea = np.ascontiguousarray(ea, dtype=np.uint8)
+    ew = np.ascontiguousarray(ew, dtype=np.uint8)
+    M, K = qa.shape
+    N = qw.shape[0]
+    assert K % MX_BLOCK == 0 and qw.shape[1] == K
+    assert ea.shape == (M, K // MX_BLOCK) and ew.shape == (N, K // MX_BLOCK)
+    rows = np.arange(M, dtype=np.int64) if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    y = np.empty((rows.size, N), dtype=np.float64)
+    b = np.empty((rows.size, N), dtype=np.float64)
+
+    def part(i0, i1):
+        lib().orc_mx_gemm_rows(_ptr(qa), _ptr(ea), _ptr(qw), _ptr(ew), N, K, _ptr(rows) + i0 * 8, i1 - i0,
+                               _ptr(y) + i0 * N * 8, _ptr(b) + i0 * N * 8)
 
     _run_parallel(part, _split(rows.size, threads), threads)
     return y, b

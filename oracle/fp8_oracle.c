@@ -22,6 +22,9 @@
  *       channels, then fp8_gemm(x, scale, weight, weight.scale)).
  *  [P5] "量化：FP8 与混合精度推理" (charles2530.github.io), "FP8 也需要 scale":
  *       x_fp8 = FP8Cast(x / s), x_hat = s * x_fp8.
+ *  [P1] section 1.2 also fixes the microscaling variant: MXFP8 splits a tensor
+ *       into blocks of 32 elements, each with its own scale factor, and the
+ *       format table of section 1.1 lists MXFP8 as 8 bits plus a shared exponent.
  *
  * Readings taken where the pages are silent or disagree (scale direction: [P3]
  * and [P5] divide where [P2] multiplies; the rest is not stated on any page):
@@ -311,4 +314,69 @@ uint16_t orc_round_bf16(double v)
     if (out > 0x1.FEp127) return sign | 0x7F80;   /* overflow -> Inf */
     c.f = (float)out;                      /* exact: out is a bf16 value */
     return (uint16_t)(sign | (c.u >> 16));
+}
+
+/* ------------------------------------------------------------- MXFP8 ([P1] 1.2) */
+
+/* Value of an E8M0 shared-exponent byte: 2^(b - 127); the byte 0xFF is NaN.
+ * (An E8M0 number has 8 exponent bits, no sign and no mantissa.) */
+double orc_e8m0_decode(uint8_t b)
+{
+    if (b == 0xFF) return NAN;
+    return ldexp(1.0, (int)b - 127);
+}
+
+/* MXFP8 quantisation of bf16 x [M][ldx] in blocks of `block` (32) consecutive
+ * elements of a row ([P1] 1.2: 32-element blocks with their own scale; 1.1: a
+ * shared exponent).  The pages do not say how the shared exponent follows from
+ * the block; the reading taken is the power-of-two rule the pages fix for
+ * scale_fmt ue8m0 ([P4]), applied per block: s = 2^ceil(log2(amax / Fmax)),
+ * e >= -126, so that no element saturates.  The exponent is stored as the E8M0
+ * byte e + 127 in e8 [M][ceil(K/block)]; codes are the cast of x / s. */
+void orc_mx_quant(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, int64_t block,
+                  int fmt, uint8_t *q, uint8_t *e8)
+{
+    int64_t nb = (K + block - 1) / block;
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t g = 0; g < nb; ++g) {
+            int64_t k0 = g * block, k1 = k0 + block < K ? k0 + block : K;
+            float amax = 0.0f;
+            for (int64_t k = k0; k < k1; ++k)
+                amax = amax_accum(amax, bf16_to_f32(x[m * ldx + k]));
+            float sc = orc_scale_from_amax(amax, fmt, ORC_SCALE_UE8M0);
+            int p;
+            double mant = frexp((double)sc, &p);   /* sc = 0.5 * 2^p exactly */
+            (void)mant;
+            e8[m * nb + g] = (uint8_t)(p - 1 + 127);
+            for (int64_t k = k0; k < k1; ++k)
+                q[m * K + k] = orc_encode(bf16_to_f32(x[m * ldx + k]) / sc, fmt);
+        }
+    }
+}
+
+/* MXFP8 GEMM, selected rows: every element of either operand carries the E8M0
+ * scale of its own 32-element block along K,
+ *   y[m][n] = sum_k dec(qa[m][k]) 2^(ea[m][k/32]-127) * dec(qw[n][k]) 2^(ew[n][k/32]-127)
+ * summed in fp64 in k order; bound[m][n] = sum_k |a_k w_k|.  qa [.][K], ea
+ * [.][K/32], qw [N][K], ew [N][K/32], K % 32 == 0. */
+void orc_mx_gemm_rows(const uint8_t *qa, const uint8_t *ea, const uint8_t *qw, const uint8_t *ew,
+                      int64_t N, int64_t K, const int64_t *rows, int64_t nr,
+                      double *y, double *bound)
+{
+    const int64_t nb = K / 32;
+    const double *dec = e4m3_values();
+    for (int64_t i = 0; i < nr; ++i) {
+        int64_t m = rows[i];
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0, b = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                double a = dec[qa[m * K + k]] * orc_e8m0_decode(ea[m * nb + k / 32]);
+                double w = dec[qw[n * K + k]] * orc_e8m0_decode(ew[n * nb + k / 32]);
+                acc += a * w;
+                b += fabs(a * w);
+            }
+            y[i * N + n] = acc;
+            bound[i * N + n] = b;
+        }
+    }
 }
