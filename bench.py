@@ -423,11 +423,11 @@ def host_cores():
 
 def cpu_baseline_prefill(S, dev):
     """The oracle as it stands (plain C, fp64 GEMM) on bounded samples of the workloads,
-    on the host cores (about 15-25 s of host time):
+    on the host cores (about 10 s of host time on a 16-core host):
       - GEMM: a few prefill rows against all 28672 weight rows, single-threaded and
         split over every usable core; full-size times are extrapolated from the
         measured fp64 MAC/s (labelled as such);
-      - act_quant: a 1024 x 7168 sweep tensor single-threaded and the full 16384 x 7168
+      - act_quant: a 4096 x 7168 sweep tensor single-threaded and the full 16384 x 7168
         sweep tensor over every usable core (Student-t(3) entries, fp32 scales)."""
     import oracle as O
     import synth
@@ -435,14 +435,14 @@ def cpu_baseline_prefill(S, dev):
     usable, reported = host_cores()
     qw = S["qw"].cpu().numpy()
     sw = S["sw"].cpu().numpy()
-    x = S["x"][: max(2, usable)].cpu()
+    rows_mt = 4 * usable                  # about 4 s of work on every core
+    x = S["x"][:rows_mt].cpu()
     qa, sa = O.act_quant(x)
 
     t = time.perf_counter()
-    O.gemm_rows(qa, sa, qw, sw, rows=[0])
+    O.gemm_rows(qa, sa, qw, sw, rows=[0, 1, 2])
     t1 = time.perf_counter() - t
-    mac1 = N * K / t1
-    rows_mt = usable
+    mac1 = 3 * N * K / t1
     t = time.perf_counter()
     O.gemm_rows(qa, sa, qw, sw, rows=list(range(rows_mt)), threads=usable)
     tmt = time.perf_counter() - t
@@ -452,7 +452,7 @@ def cpu_baseline_prefill(S, dev):
     xs = synth.activations(16384, 7168, seed=0, dist="t3", device=dev).cpu()
     aq_bytes = lambda m: m * 7168 * 3 + m * 56 * 4
     t = time.perf_counter()
-    O.act_quant(xs[:1024])
+    O.act_quant(xs[:4096])
     taq1 = time.perf_counter() - t
     t = time.perf_counter()
     O.act_quant(xs, threads=usable)
@@ -460,13 +460,13 @@ def cpu_baseline_prefill(S, dev):
     return {"value": round(2.0 * macmt / 1e12, 6), "unit": "TFLOPS", "cores": usable, "kind": "oracle",
             "host_cores": reported,
             "sample": f"fp64 GEMM of {rows_mt} prefill rows x {N} x {K} split over {usable} threads "
-                      f"(plus 1 row single-threaded); act_quant of the 16384x7168 sweep tensor over {usable} "
-                      f"threads and of 1024x7168 single-threaded",
+                      f"(plus 3 rows single-threaded); act_quant of the 16384x7168 sweep tensor over {usable} "
+                      f"threads and of 4096x7168 single-threaded",
             "gemm": {"mac_per_s_1thread": round(mac1), "mac_per_s_all_cores": round(macmt),
                      "prefill_full_s_extrapolated_1thread": round(full_mac / mac1, 1),
                      "prefill_full_s_extrapolated_all_cores": round(full_mac / macmt, 1),
                      "TFLOPS_1thread": round(2.0 * mac1 / 1e12, 6)},
-            "act_quant": {"GB/s_1thread (1024x7168)": round(aq_bytes(1024) / taq1 / 1e9, 3),
+            "act_quant": {"GB/s_1thread (4096x7168)": round(aq_bytes(4096) / taq1 / 1e9, 3),
                           "GB/s_all_cores (16384x7168)": round(aq_bytes(16384) / taqmt / 1e9, 3),
                           "s_all_cores (16384x7168)": round(taqmt, 2)},
             "seconds": round(t1 + tmt + taq1 + taqmt, 2)}
