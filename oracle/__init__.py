@@ -59,6 +59,9 @@ def lib():
         L.orc_mx_quant.argtypes = [vp, i64, i64, i64, i64, ctypes.c_int, vp, vp]
         L.orc_mx_gemm_rows.restype = None
         L.orc_mx_gemm_rows.argtypes = [vp, vp, vp, vp, i64, i64, vp, i64, vp, vp]
+        L.orc_delayed_quant.restype = None
+        L.orc_delayed_quant.argtypes = [vp, i64, ctypes.c_int, ctypes.c_float, i64, ctypes.c_int, vp, vp, vp, vp,
+                                        vp, vp]
         L.orc_grouped_gemm_rows.restype = None
         L.orc_grouped_gemm_rows.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp, i64, vp, vp]
         del u8p
@@ -283,3 +286,29 @@ def mx_gemm_rows(qa, ea, qw, ew, rows=None, threads: int = 1):
 
     _run_parallel(part, _split(rows.size, threads), threads)
     return y, b
+
+
+# ------------------------------------------------------- delayed scaling
+ALGO_MOST_RECENT, ALGO_MAX = 0, 1
+
+
+class DelayedScalingState:
+    """Host copy of the delayed-scaling state: the scale for the next step (starts at
+    1.0), the history ring of past amaxes and the slot the next amax goes to."""
+
+    def __init__(self, hist_len: int = 16):
+        self.scale = np.array([1.0], np.float32)
+        self.pos = np.array([0], np.int32)
+        self.history = np.zeros(hist_len, np.float32)
+
+
+def delayed_quant(x, state: DelayedScalingState, fmt: int = E4M3, target: float = 400.0, algo: int = ALGO_MAX):
+    """One step: codes of x under the previous step's scale, the number of clipped
+    elements, the scale used; `state` is updated in place for the next step."""
+    xb = _bf16_bits(x)
+    q = np.empty(xb.shape, dtype=np.uint8)
+    n_clip = np.zeros(1, np.uint64)
+    s_used = np.zeros(1, np.float32)
+    lib().orc_delayed_quant(_ptr(xb), xb.size, fmt, float(target), state.history.size, algo, _ptr(state.scale),
+                            _ptr(state.pos), _ptr(state.history), _ptr(q), _ptr(n_clip), _ptr(s_used))
+    return q, int(n_clip[0]), float(s_used[0])

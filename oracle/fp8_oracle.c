@@ -380,3 +380,49 @@ void orc_mx_gemm_rows(const uint8_t *qa, const uint8_t *ea, const uint8_t *qw, c
         }
     }
 }
+
+/* ----------------------------------------------- delayed scaling ([P1] 4.3, 6) */
+
+/* One step of delayed per-tensor scaling as the ROCm/AITER page describes it
+ * ([P1] 4.3 "延迟缩放", the FP8DelayedScaling listing; [P1] section 6, amax history
+ * length and "max" over the history):
+ *   1. the tensor is divided by the scale of the PREVIOUS step (*scale; the page
+ *      starts from 1.0), clamped to +-Fmax and cast -- q[i] = enc(x[i] / s_prev);
+ *      elements whose quotient lies beyond +-Fmax are the clipped ones the page's
+ *      checklist asks to count ("FP8 溢出率": *n_clipped);
+ *   2. the current amax max|x| goes into the history ring at slot *pos;
+ *   3. the next step's scale is (max over the history if algo == 1, else the amax
+ *      just recorded) / target, target = 400 for E4M3 on the page (a margin below
+ *      448), floored at 2^-126 (reading shared with the other quantisers: a zero
+ *      amax must not give a zero divisor); the slot after *pos is cleared for the
+ *      next step and *pos advances.
+ * *s_used receives the scale the codes were made with (x ~= dec(q) * s_used).
+ * The history holds non-negative amaxes; zeros are slots not yet filled. */
+void orc_delayed_quant(const uint16_t *x, int64_t n, int fmt, float target, int64_t hist_len,
+                       int algo, float *scale, int32_t *pos, float *history,
+                       uint8_t *q, uint64_t *n_clipped, float *s_used)
+{
+    const double fmax = orc_fmax(fmt);
+    const float s_prev = *scale;
+    uint64_t clipped = 0;
+    float amax = 0.0f;
+    for (int64_t i = 0; i < n; ++i) {
+        float v = bf16_to_f32(x[i]);
+        float t = v / s_prev;                  /* one IEEE division */
+        if (fabs((double)t) > fmax) ++clipped;
+        q[i] = orc_encode(t, fmt);             /* clamp to +-Fmax, then round */
+        amax = amax_accum(amax, v);
+    }
+    *n_clipped = clipped;
+    *s_used = s_prev;
+    int32_t p = *pos;
+    history[p] = amax;
+    float a = amax;
+    if (algo == 1)
+        for (int64_t h = 0; h < hist_len; ++h) a = history[h] > a ? history[h] : a;
+    float s_next = a / target;
+    *scale = s_next < 0x1p-126f ? 0x1p-126f : s_next;
+    p = (int32_t)((p + 1) % hist_len);
+    history[p] = 0.0f;
+    *pos = p;
+}
