@@ -409,6 +409,76 @@ def measure_rows(dev, peaks):
                                                     "GB/s": round(b / ms / 1e6, 1),
                                                     "frac_hbm": round(b / ms / 1e6 / hbm, 4)}
     assert F.fp8_device_error() == 0
+    del qwe, swe, qa, sa, y
+    res.update(measure_mx_rows(dev, peaks))
+    return res
+
+
+def measure_mx_rows(dev, peaks):
+    """The tensor core's scale path: MXFP8 quantisation and GEMM (32-element E8M0
+    blocks), and the ue8m0 (power-of-two) configurations on it."""
+    import torch
+    import fp8_block_scaled_12_b200 as F
+    import synth
+    res = {}
+    hbm = peaks["hbm_gbs"]
+    fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
+    x = synth.activations(16384, 7168, seed=0, dist="t3", device=dev)
+    q = torch.empty(x.shape, dtype=torch.uint8, device=dev)
+    e8 = torch.empty((F.mx_sf_bytes(16384, 7168),), dtype=torch.uint8, device=dev)
+    ms = time_launches(lambda: F.fp8_mx_quant(x, q, e8), 20)
+    b = x.numel() * 3 + x.numel() // 32
+    res["mx_quant 16384x7168"] = {"GB/s": round(b / ms / 1e6, 1), "frac_hbm": round(b / ms / 1e6 / hbm, 4)}
+    del x, q, e8
+    # prefill shape: MXFP8 (32-element exponents) and the ue8m0 scales (128 / 128x128) packed
+    p = synth.PREFILL.params
+    M, N, K = p["M"], p["N"], p["K"]
+    xa = synth.activations(M, K, seed=0, device=dev)
+    w = synth.weights(N, K, p["w_std"], seed=0, device=dev)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    fl = 2.0 * M * N * K
+    qa, ea = F.mx_quant(xa)
+    qw, ew = F.mx_quant(w)
+    ms = time_launches(lambda: F.fp8_mx_gemm(qa, ea, qw, ew, y), 10)
+    res["mx_gemm e8m0x32 prefill 4096x28672x8192"] = {"us": round(ms * 1e3, 1), "TFLOPS": round(fl / ms / 1e9, 1),
+                                                       "frac_fp8_peak": round(fl / ms / 1e9 / fp8_peak, 4)}
+    qa, sa = F.act_quant(xa, scale_fmt=F.SCALE_UE8M0)
+    qw, sw = F.weight_quant(w, scale_fmt=F.SCALE_UE8M0)
+    del w
+    ew = F.mx_pack_pow2(sw, N, K, 128)                       # weights: once
+    ea = torch.empty((F.mx_sf_bytes(M, K),), dtype=torch.uint8, device=dev)
+
+    def pow2_step():                                         # activations: every call
+        F.fp8_mx_pack_pow2(sa, M, K, 1, ea)
+        F.fp8_mx_gemm(qa, ea, qw, ew, y)
+
+    ms = time_launches(pow2_step, 10)
+    res["mx_gemm ue8m0 prefill 4096x28672x8192 (pack + gemm)"] = {
+        "us": round(ms * 1e3, 1), "TFLOPS": round(fl / ms / 1e9, 1), "frac_fp8_peak": round(fl / ms / 1e9 / fp8_peak, 4)}
+    ms = time_launches(lambda: F.fp8_block_gemm(qa, sa, qw, sw, y), 10)
+    res["block_gemm (promotion) ue8m0 prefill 4096x28672x8192"] = {
+        "us": round(ms * 1e3, 1), "TFLOPS": round(fl / ms / 1e9, 1), "frac_fp8_peak": round(fl / ms / 1e9 / fp8_peak, 4)}
+    del qa, sa, qw, sw, xa, y, ea, ew
+    # decode config (ue8m0) on the scale path: weights packed once, activations per call
+    wd = synth.weights(18432, 7168, 0.015, seed=0, device=dev)
+    qwd, swd = F.weight_quant(wd, scale_fmt=F.SCALE_UE8M0)
+    del wd
+    ewd = F.mx_pack_pow2(swd, 18432, 7168, 128)
+    for Md in (1, 64):
+        xd = synth.activations(Md, 7168, seed=0, device=dev)
+        qa, sa = F.act_quant(xd, scale_fmt=F.SCALE_UE8M0)
+        ea = torch.empty((F.mx_sf_bytes(Md, 7168),), dtype=torch.uint8, device=dev)
+        y = torch.empty((Md, 18432), dtype=torch.bfloat16, device=dev)
+
+        def dstep():
+            F.fp8_mx_pack_pow2(sa, Md, 7168, 1, ea)
+            F.fp8_mx_gemm(qa, ea, qwd, ewd, y)
+
+        ms = time_launches(dstep, 20)
+        b = 18432 * 7168 + ewd.numel() + Md * (7168 + 56 * 4 + 18432 * 2)
+        res[f"mx_gemm ue8m0 decode M={Md} (pack + gemm)"] = {"us": round(ms * 1e3, 2), "GB/s": round(b / ms / 1e6, 1),
+                                                            "frac_hbm": round(b / ms / 1e6 / hbm, 4)}
+    assert F.fp8_device_error() == 0
     return res
 
 

@@ -20,19 +20,22 @@ import torch
 
 __all__ = [
     "E4M3", "E5M2", "SCALE_FP32", "SCALE_UE8M0", "OUT_BF16", "OUT_FP32", "Fp8Error", "LIB_PATH",
-    "fp8_act_quant", "fp8_weight_quant", "fp8_block_gemm", "fp8_grouped_gemm",
-    "fp8_status_string", "fp8_device_error", "fp8_selftest_bounded_wait",
-    "act_quant", "weight_quant", "block_gemm", "grouped_gemm", "EXPORTS",
+    "fp8_act_quant", "fp8_weight_quant", "fp8_block_gemm", "fp8_grouped_gemm", "fp8_mx_quant", "fp8_mx_gemm",
+    "fp8_mx_pack_pow2", "fp8_status_string", "fp8_device_error", "fp8_selftest_bounded_wait",
+    "act_quant", "weight_quant", "block_gemm", "grouped_gemm", "mx_quant", "mx_gemm", "mx_pack_pow2",
+    "mx_sf_bytes", "EXPORTS",
 ]
 
 E4M3, E5M2 = 0, 1
 SCALE_FP32, SCALE_UE8M0 = 0, 1
 OUT_BF16, OUT_FP32 = 0, 1
+MX_BLOCK = 32
 FP8_OK = 0
+FP8_ERR_INVALID_SCALE = 7
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfp8lin.so")
-EXPORTS = ("fp8_act_quant", "fp8_weight_quant", "fp8_block_gemm", "fp8_grouped_gemm",
-           "fp8_status_string", "fp8_device_error", "fp8_selftest_bounded_wait")
+EXPORTS = ("fp8_act_quant", "fp8_weight_quant", "fp8_block_gemm", "fp8_grouped_gemm", "fp8_mx_quant",
+           "fp8_mx_gemm", "fp8_mx_pack_pow2", "fp8_status_string", "fp8_device_error", "fp8_selftest_bounded_wait")
 
 
 class Fp8Error(RuntimeError):
@@ -50,12 +53,15 @@ def _load() -> ctypes.CDLL:
     L.fp8_weight_quant.argtypes = [vp, i64, i64, ci, ci, ci, vp, vp, vp]
     L.fp8_block_gemm.argtypes = [vp, vp, vp, vp, i64, i64, i64, ci, vp, vp]
     L.fp8_grouped_gemm.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, ci, vp, vp]
+    L.fp8_mx_quant.argtypes = [vp, i64, i64, i64, ci, vp, vp, vp]
+    L.fp8_mx_gemm.argtypes = [vp, vp, vp, vp, i64, i64, i64, ci, vp, vp]
+    L.fp8_mx_pack_pow2.argtypes = [vp, i64, i64, ci, vp, vp]
     L.fp8_status_string.argtypes = [ci]
     L.fp8_status_string.restype = ctypes.c_char_p
     L.fp8_device_error.argtypes = [vp]
     L.fp8_selftest_bounded_wait.argtypes = [i64, vp]
-    for name in ("fp8_act_quant", "fp8_weight_quant", "fp8_block_gemm", "fp8_grouped_gemm", "fp8_device_error",
-                 "fp8_selftest_bounded_wait"):
+    for name in ("fp8_act_quant", "fp8_weight_quant", "fp8_block_gemm", "fp8_grouped_gemm", "fp8_mx_quant",
+                 "fp8_mx_gemm", "fp8_mx_pack_pow2", "fp8_device_error", "fp8_selftest_bounded_wait"):
         getattr(L, name).restype = ci
     return L
 
@@ -185,6 +191,50 @@ def fp8_grouped_gemm(qa: torch.Tensor, sa: torch.Tensor, qw: torch.Tensor, sw: t
                                                     _stream(stream)))
 
 
+def mx_sf_bytes(rows: int, K: int) -> int:
+    """Bytes of the tiled MXFP8 exponent layout of a [rows, K] operand (FP8_MX_SF_BYTES)."""
+    return ((rows + 127) // 128) * ((K + 127) // 128) * 512
+
+
+def fp8_mx_quant(x: torch.Tensor, q: torch.Tensor, e8: torch.Tensor, fmt: int = E4M3, stream=None) -> None:
+    """MXFP8 quantisation of bf16 x [M, K] (row stride x.stride(0)) into codes q [M, K]
+    and E8M0 exponent bytes e8 (uint8, mx_sf_bytes(M, K), tiled layout of the header)."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    assert q.is_contiguous() and e8.is_contiguous()
+    M, K = x.shape
+    _expect(q, (M, K), "q")
+    _expect(e8, (mx_sf_bytes(M, K),), "e8", torch.uint8)
+    _check("fp8_mx_quant", lib.fp8_mx_quant(_ptr(x), M, K, x.stride(0), fmt, _ptr(_u8(q)), _ptr(e8),
+                                            _stream(stream)))
+
+
+def fp8_mx_gemm(qa: torch.Tensor, sfa: torch.Tensor, qw: torch.Tensor, sfw: torch.Tensor, y: torch.Tensor,
+                stream=None) -> None:
+    """y [M, N] = FP8 GEMM with E8M0 scales per 32-element block of K applied by the
+    tensor core; sfa / sfw are tiled exponent bytes (mx_quant, or mx_pack_pow2 for the
+    ue8m0 scales of act_quant / weight_quant)."""
+    for t in (qa, sfa, qw, sfw, y):
+        assert t.is_contiguous()
+    M, K = qa.shape
+    N = qw.shape[0]
+    _expect(qw, (N, K), "qw")
+    _expect(sfa, (mx_sf_bytes(M, K),), "sfa", torch.uint8)
+    _expect(sfw, (mx_sf_bytes(N, K),), "sfw", torch.uint8)
+    _expect(y, (M, N), "y")
+    qa8, qw8, od = _e4m3_codes(qa, "qa"), _e4m3_codes(qw, "qw"), _out_code(y)
+    _check("fp8_mx_gemm", lib.fp8_mx_gemm(_ptr(qa8), _ptr(sfa), _ptr(qw8), _ptr(sfw), M, N, K, od, _ptr(y),
+                                          _stream(stream)))
+
+
+def fp8_mx_pack_pow2(s: torch.Tensor, rows: int, K: int, row_block: int, sf: torch.Tensor, stream=None) -> None:
+    """fp32 power-of-two scales in the block GEMM's layout (row_block 1: [rows, K/128];
+    128: [ceil(rows/128), K/128]) -> tiled exponent bytes sf (mx_sf_bytes(rows, K))."""
+    assert s.dtype == torch.float32 and s.is_contiguous() and sf.is_contiguous()
+    _expect(s, (rows if row_block == 1 else (rows + 127) // 128, K // 128), "s")
+    _expect(sf, (mx_sf_bytes(rows, K),), "sf", torch.uint8)
+    _check("fp8_mx_pack_pow2", lib.fp8_mx_pack_pow2(_ptr(s), rows, K, row_block, _ptr(sf), _stream(stream)))
+
+
 def fp8_device_error(stream=None) -> int:
     """Synchronise the stream and return (and clear) the device-side wait status."""
     return int(lib.fp8_device_error(_stream(stream)))
@@ -225,3 +275,23 @@ def grouped_gemm(qa, sa, qw, sw, offsets, out_dtype=torch.bfloat16, stream=None)
     y = torch.empty((qa.shape[0], qw.shape[1]), dtype=out_dtype, device=qa.device)
     fp8_grouped_gemm(qa, sa, qw, sw, offsets, y, stream)
     return y
+
+
+def mx_quant(x: torch.Tensor, fmt: int = E4M3, stream=None):
+    M, K = x.shape
+    q = torch.empty((M, K), dtype=torch.uint8, device=x.device)
+    e8 = torch.empty((mx_sf_bytes(M, K),), dtype=torch.uint8, device=x.device)
+    fp8_mx_quant(x, q, e8, fmt, stream)
+    return q, e8
+
+
+def mx_gemm(qa, sfa, qw, sfw, out_dtype=torch.bfloat16, stream=None):
+    y = torch.empty((qa.shape[0], qw.shape[0]), dtype=out_dtype, device=qa.device)
+    fp8_mx_gemm(qa, sfa, qw, sfw, y, stream)
+    return y
+
+
+def mx_pack_pow2(s: torch.Tensor, rows: int, K: int, row_block: int, stream=None):
+    sf = torch.empty((mx_sf_bytes(rows, K),), dtype=torch.uint8, device=s.device)
+    fp8_mx_pack_pow2(s, rows, K, row_block, sf, stream)
+    return sf

@@ -9,6 +9,7 @@
 
 #include "../../include/fp8lin.h"
 #include "gemm.cuh"
+#include "gemm_mx.cuh"
 #include "gemm_swap.cuh"
 #include "ptx.cuh"
 #include "quant.cuh"
@@ -103,6 +104,31 @@ int launch_swap(const void* qa, const void* qw, const GemmArgs& a, int64_t w_row
   return cuda_status(cudaGetLastError());
 }
 
+// Block-scaled (power-of-two) GEMM on the tensor core's scale path.  WIDE: P = 128
+// activation rows, Q = 256 weight rows; SWAP (few tokens): P = 128 weight rows, Q =
+// up to NQ tokens in 32-row boxes.
+template <bool SWAP, int NQ, int STAGES>
+int launch_mx(const void* qa, const void* qw, const MxArgs& a, cudaStream_t st) {
+  using C = MxCfg<SWAP, NQ, STAGES>;
+  constexpr size_t smem = mx_smem_bytes<C>();
+  static_assert(smem <= 232448, "dynamic shared memory of one CTA (227 KB)");
+  CUtensorMap mp, mq;
+  const void* pp = SWAP ? qw : qa;
+  const void* qp = SWAP ? qa : qw;
+  const uint64_t prow = uint64_t(SWAP ? a.N : a.M), qrow = uint64_t(SWAP ? a.M : a.N);
+  if (!make_map_u8(&mp, pp, prow, uint64_t(a.K), 128)) return FP8_ERR_CUDA;
+  if (!make_map_u8(&mq, qp, qrow, uint64_t(a.K), SWAP ? 32u : uint32_t(NQ))) return FP8_ERR_CUDA;
+  auto kern = k_gemm_mx<C>;
+  if (!launch_regs_ok(kern)) return FP8_ERR_UNSUPPORTED;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return FP8_ERR_CUDA;
+  const int64_t tiles = SWAP ? int64_t((a.N + 127) / 128) * ((a.M + NQ - 1) / NQ)
+                             : int64_t((a.M + 127) / 128) * ((a.N + NQ - 1) / NQ);
+  const int grid = int(tiles < num_sms() ? tiles : num_sms());
+  kern<<<grid, kThreads, smem, st>>>(mp, mq, a);
+  return cuda_status(cudaGetLastError());
+}
+
 int launch_wide(const void* qa, const void* qw, const GemmArgs& a, cudaStream_t st) {
   using C = WideCfg<kWideStages>;
   CUtensorMap ma, mb;
@@ -134,6 +160,20 @@ int launch_act_quant(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, uint8
   const int64_t warps = (steps + per_warp - 1) / per_warp;
   const int64_t blocks = (warps + 7) / 8;
   k_act_quant<FMT, SF, U><<<int(blocks), 256, 0, st>>>(x, M, K, ldx, q, s);
+  return cuda_status(cudaGetLastError());
+}
+
+template <int FMT>
+int launch_mx_quant(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q, uint8_t* e8,
+                    cudaStream_t st) {
+  constexpr int U = 2;
+  const int64_t items = M * ((K + 127) / 128);
+  const int64_t steps = (items + 8 * U - 1) / (8 * U);
+  const int64_t max_warps = int64_t(num_sms()) * 8 * (256 / 32);
+  const int64_t per_warp = (steps + max_warps - 1) / max_warps;
+  const int64_t warps = (steps + per_warp - 1) / per_warp;
+  const int64_t blocks = (warps + 7) / 8;
+  k_act_quant<FMT, kScaleUe8m0, U, true><<<int(blocks), 256, 0, st>>>(x, M, K, ldx, q, e8);
   return cuda_status(cudaGetLastError());
 }
 
@@ -192,6 +232,7 @@ const char* fp8_status_string(int status) {
     case FP8_ERR_UNSUPPORTED: return "unsupported option";
     case FP8_ERR_CUDA: return "CUDA error";
     case FP8_ERR_TIMEOUT: return "device wait timed out";
+    case FP8_ERR_INVALID_SCALE: return "a scale given as a power of two is not one";
     default: return "unknown status";
   }
 }
@@ -283,6 +324,53 @@ int fp8_grouped_gemm(const void* qa, const float* sa, const void* qw, const floa
   return launch_swap<160, 3, 5, 28>(qa, qw, a, E * N, static_cast<cudaStream_t>(stream));
 }
 
+int fp8_mx_quant(const void* x, int64_t M, int64_t K, int64_t ldx, int fmt, void* q, void* e8, void* stream) {
+  if (M < 0 || K <= 0 || ldx < K) return FP8_ERR_INVALID_ARG;
+  if (fmt != FP8_E4M3 && fmt != FP8_E5M2) return FP8_ERR_INVALID_ARG;
+  if (K % 16 != 0) return FP8_ERR_SHAPE;
+  if (M == 0) return FP8_OK;
+  if (!x || !q || !e8) return FP8_ERR_INVALID_ARG;
+  if (ldx % 8 != 0 || !aligned(x, 16) || !aligned(q, 16)) return FP8_ERR_ALIGNMENT;
+  const uint16_t* xb = static_cast<const uint16_t*>(x);
+  uint8_t* qb = static_cast<uint8_t*>(q);
+  uint8_t* eb = static_cast<uint8_t*>(e8);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return fmt == FP8_E4M3 ? launch_mx_quant<kE4M3>(xb, M, K, ldx, qb, eb, st)
+                         : launch_mx_quant<kE5M2>(xb, M, K, ldx, qb, eb, st);
+}
+
+int fp8_mx_gemm(const void* qa, const void* sfa, const void* qw, const void* sfw, int64_t M, int64_t N,
+                int64_t K, int out_dtype, void* y, void* stream) {
+  if (M < 0 || N <= 0 || K <= 0) return FP8_ERR_INVALID_ARG;
+  if (out_dtype != FP8_OUT_BF16 && out_dtype != FP8_OUT_FP32) return FP8_ERR_INVALID_ARG;
+  if (K % 128 != 0 || N % 16 != 0) return FP8_ERR_SHAPE;
+  if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return FP8_ERR_SHAPE;
+  if (!qw || !sfw) return FP8_ERR_INVALID_ARG;
+  if (M > 0 && (!qa || !sfa || !y)) return FP8_ERR_INVALID_ARG;
+  if (!aligned(qw, 16) || !aligned(sfw, 16)) return FP8_ERR_ALIGNMENT;
+  if (M > 0 && (!aligned(qa, 16) || !aligned(sfa, 16) || !aligned(y, 16))) return FP8_ERR_ALIGNMENT;
+  if (M == 0) return FP8_OK;
+  MxArgs a{static_cast<const uint8_t*>(sfa), static_cast<const uint8_t*>(sfw), y, int(M), int(N), int(K),
+           out_dtype == FP8_OUT_FP32 ? 1 : 0};
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (M <= 64) return launch_mx<true, 64, 8>(qa, qw, a, st);
+  if (M <= 160) return launch_mx<true, 160, 5>(qa, qw, a, st);
+  return launch_mx<false, 256, 4>(qa, qw, a, st);
+}
+
+int fp8_mx_pack_pow2(const float* s, int64_t rows, int64_t K, int row_block, void* sf, void* stream) {
+  if (rows < 0 || K <= 0) return FP8_ERR_INVALID_ARG;
+  if (row_block != 1 && row_block != 128) return FP8_ERR_INVALID_ARG;
+  if (K % 128 != 0) return FP8_ERR_SHAPE;
+  if (rows == 0) return FP8_OK;
+  if (!s || !sf) return FP8_ERR_INVALID_ARG;
+  if (!aligned(s, 4) || !aligned(sf, 16)) return FP8_ERR_ALIGNMENT;
+  const int64_t nkb = K / 128, n = rows * nkb;
+  k_mx_pack_pow2<<<unsigned((n + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      s, rows, nkb, row_block, static_cast<uint8_t*>(sf));
+  return cuda_status(cudaGetLastError());
+}
+
 int fp8_selftest_bounded_wait(int64_t limit_ns, void* stream) {
   if (limit_ns <= 0 || limit_ns > 10000000000ll) return FP8_ERR_INVALID_ARG;
   k_selftest_wait<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(uint64_t(limit_ns));
@@ -295,7 +383,9 @@ int fp8_device_error(void* stream) {
   unsigned int v = 0, zero = 0;
   if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v)) != cudaSuccess) return FP8_ERR_CUDA;
   if (v != 0 && cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess) return FP8_ERR_CUDA;
-  return v ? FP8_ERR_TIMEOUT : FP8_OK;
+  if (v & 1u) return FP8_ERR_TIMEOUT;
+  if (v & kErrBadScale) return FP8_ERR_INVALID_SCALE;
+  return FP8_OK;
 }
 
 }  // extern "C"

@@ -139,16 +139,33 @@ __device__ __forceinline__ uint4 ldg_stream(const uint4* p) {
   return r;
 }
 
+// Byte offset of the E8M0 exponent of (row r, 32-element block g) in the tiled scale
+// layout the block-scaled MMA reads (gemm_mx.cuh): 512-byte atoms of 128 rows x 4
+// blocks, atom (r / 128, g / 4) at (r / 128 * nkb + g / 4) * 512, nkb = ceil(K / 128);
+// inside it (r % 32) * 16 + (r % 128 / 32) * 4 + g % 4.
+__host__ __device__ __forceinline__ int64_t mx_tiled_offset(int64_t r, int64_t g, int64_t nkb) {
+  const int64_t rb = r >> 7, rr = r & 127, kb = g >> 2, j = g & 3;
+  return (rb * nkb + kb) * 512 + (rr & 31) * 16 + (rr >> 5) * 4 + j;
+}
+
 // ---------------------------------------------------------------- act_quant
 // Work item = (row m, group g) of 128 channels, owned by 4 consecutive lanes: lane
 // quarter t holds channels [32t, 32t+32) of the group (four 16-byte loads), so the
 // group amax needs two shuffles and each lane casts 32 values with one scale.  A
 // warp takes 8 consecutive items per step (consecutive groups of a row are adjacent
 // in memory: a 2 KB contiguous span), and UNROLL steps per loop iteration.
-template <int FMT, int SF, int UNROLL>
+//
+// MX = true is the MXFP8 variant ("ROCm 7 ... AITER", section 1.2: blocks of 32
+// elements, each with its own scale; section 1.1: a shared exponent): each lane's 32
+// channels are one block, so the block amax needs no shuffle; the scale follows the
+// ue8m0 rule and is stored as its E8M0 byte (the fp32 exponent field of the power of
+// two) in s_out, in the tiled layout of mx_tiled_offset.  Otherwise s_out = fp32
+// [M][ceil(K/128)].
+template <int FMT, int SF, int UNROLL, bool MX = false>
 __global__ void __launch_bounds__(256) k_act_quant(const uint16_t* __restrict__ x, int64_t M,
                                                    int64_t K, int64_t ldx, uint8_t* __restrict__ q,
-                                                   float* __restrict__ s) {
+                                                   void* __restrict__ s_out) {
+  static_assert(!MX || SF == kScaleUe8m0, "MXFP8 exponents follow the ue8m0 rule");
   const int64_t ng = (K + 127) / 128;
   const int64_t total = M * ng;
   const int lane = threadIdx.x & 31;
@@ -183,8 +200,10 @@ __global__ void __launch_bounds__(256) k_act_quant(const uint16_t* __restrict__ 
       float a = 0.0f;
 #pragma unroll
       for (int j = 0; j < 4; ++j) a = amax8(v[u][j], a);
-      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
-      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+      if (!MX) {
+        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+      }
       const GroupScale<FMT, SF> sc(a);
       if (item_ok[u]) {
         uint8_t* dst = q + row[u] * K + col[u];
@@ -196,7 +215,13 @@ __global__ void __launch_bounds__(256) k_act_quant(const uint16_t* __restrict__ 
             *reinterpret_cast<uint4*>(dst + 16 * h) = make_uint4(lo.x, lo.y, hi.x, hi.y);
           }
         }
-        if (qt == 0) s[row[u] * ng + (col[u] >> 7)] = sc.s;
+        if (MX) {
+          if (col[u] < K)
+            static_cast<uint8_t*>(s_out)[mx_tiled_offset(row[u], col[u] >> 5, ng)] =
+                uint8_t(__float_as_uint(sc.s) >> 23);
+        } else if (qt == 0) {
+          static_cast<float*>(s_out)[row[u] * ng + (col[u] >> 7)] = sc.s;
+        }
       }
     }
   }

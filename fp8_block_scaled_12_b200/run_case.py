@@ -4,6 +4,8 @@
     python -m fp8_block_scaled_12_b200.run_case --op act_quant --M 16384 --K 7168 --scale ue8m0
     python -m fp8_block_scaled_12_b200.run_case --op weight_quant --M 28672 --K 8192 --block 0 --fmt e5m2
     python -m fp8_block_scaled_12_b200.run_case --op grouped --tokens 4096 --E 256 --N 2048 --K 7168
+    python -m fp8_block_scaled_12_b200.run_case --op mx_gemm --M 4096 --N 28672 --K 8192 --scale ue8m0
+    python -m fp8_block_scaled_12_b200.run_case --op mx_quant --M 16384 --K 7168
 
 Inputs are prepared before the measured launches (so a profiler can skip them by
 launch count: the op's own launches come last, `--iters` of them, after `--warm`
@@ -42,7 +44,8 @@ def timed(fn, warm, iters):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--op", required=True, choices=["act_quant", "weight_quant", "gemm", "grouped"])
+    ap.add_argument("--op", required=True, choices=["act_quant", "weight_quant", "gemm", "grouped", "mx_quant",
+                                                    "mx_gemm"])
     ap.add_argument("--M", type=int, default=4096)
     ap.add_argument("--N", type=int, default=28672)
     ap.add_argument("--K", type=int, default=8192)
@@ -91,6 +94,32 @@ def main():
         b = qa.numel() + qw.numel() + y.numel() * y.element_size() + sa.numel() * 4 + sw.numel() * 4
         print(f"gemm M={a.M} N={a.N} K={a.K} {a.scale} {a.out}: {ms * 1e3:.2f} us  {fl / ms / 1e9:.1f} TFLOPS  "
               f"{b / ms / 1e6:.1f} GB/s")
+    elif a.op == "mx_quant":
+        x = synth.activations(a.M, a.K, seed=0, dist=a.dist, device=dev)
+        q = torch.empty((a.M, a.K), dtype=torch.uint8, device=dev)
+        e8 = torch.empty((F.mx_sf_bytes(a.M, a.K),), dtype=torch.uint8, device=dev)
+        ms = timed(lambda: F.fp8_mx_quant(x, q, e8, fmt=fmt), a.warm, a.iters)
+        b = a.M * a.K * 3 + a.M * ((a.K + 31) // 32)
+        print(f"mx_quant M={a.M} K={a.K} {a.fmt}: {ms * 1e3:.2f} us  {b / ms / 1e6:.1f} GB/s")
+    elif a.op == "mx_gemm":
+        # --scale fp32 selects MXFP8 (32-element E8M0 exponents), ue8m0 the power-of-two
+        # scales of the block GEMM's layout
+        x = synth.activations(a.M, a.K, seed=0, device=dev)
+        w = synth.weights(a.N, a.K, 0.02, seed=0, device=dev)
+        if a.scale == "fp32":
+            qa, sa = F.mx_quant(x)
+            qw, sw = F.mx_quant(w)
+        else:
+            qa, s_a = F.act_quant(x, scale_fmt=F.SCALE_UE8M0)
+            qw, s_w = F.weight_quant(w, scale_fmt=F.SCALE_UE8M0)
+            sa = F.mx_pack_pow2(s_a, a.M, a.K, 1)
+            sw = F.mx_pack_pow2(s_w, a.N, a.K, 128)
+        del x, w
+        y = torch.empty((a.M, a.N), dtype=odt, device=dev)
+        ms = timed(lambda: F.fp8_mx_gemm(qa, sa, qw, sw, y), a.warm, a.iters)
+        fl = 2.0 * a.M * a.N * a.K
+        layout = "e8m0x32" if a.scale == "fp32" else "pow2x128"
+        print(f"mx_gemm M={a.M} N={a.N} K={a.K} {layout} {a.out}: {ms * 1e3:.2f} us  {fl / ms / 1e9:.1f} TFLOPS")
     else:
         row_token, _, off = synth.routing(a.tokens, a.E, a.topk, seed=0)
         xt = synth.activations(a.tokens, a.K, seed=0, device=dev)

@@ -45,7 +45,10 @@ typedef enum {
     FP8_ERR_ALIGNMENT = 3,     /* pointer or leading dimension misaligned        */
     FP8_ERR_UNSUPPORTED = 4,   /* valid request this build does not implement    */
     FP8_ERR_CUDA = 5,          /* a CUDA runtime call or launch failed           */
-    FP8_ERR_TIMEOUT = 6        /* a bounded device-side wait ran out             */
+    FP8_ERR_TIMEOUT = 6,       /* a bounded device-side wait ran out             */
+    FP8_ERR_INVALID_SCALE = 7  /* fp8_mx_pack_pow2 got a scale that is not a
+                                  positive normal power of two (reported by
+                                  fp8_device_error)                              */
 } fp8_status;
 
 typedef enum { FP8_E4M3 = 0, FP8_E5M2 = 1 } fp8_format;
@@ -129,6 +132,72 @@ int fp8_grouped_gemm(const void* qa, const float* sa, const void* qw, const floa
                      const int32_t* group_offsets, int64_t E, int64_t total_M,
                      int64_t N, int64_t K, int out_dtype, void* y, void* stream);
 
+/*
+ * MXFP8 scale layout ("tiled").  The exponent bytes of an operand with R rows and K
+ * columns are stored in the order the tensor core's block-scaled MMA reads them:
+ * ceil(R/128) x ceil(K/128) atoms of 512 bytes, atom (rb, kb) at byte offset
+ * (rb * ceil(K/128) + kb) * 512; inside an atom, row r (0..127 of row block rb) and
+ * 32-element block j (0..3 of K-block kb) are at byte (r % 32) * 16 + (r / 32) * 4 + j.
+ * Size in bytes: FP8_MX_SF_BYTES(R, K).  Bytes of rows >= R or of blocks beyond K are
+ * not written by fp8_mx_quant and not read for any output.
+ */
+#define FP8_MX_SF_BYTES(R, K) ((((int64_t)(R) + 127) / 128) * (((int64_t)(K) + 127) / 128) * 512)
+
+/*
+ * fp8_mx_quant -- MXFP8 quantisation ("ROCm 7 原生 FP8/MXFP8 ... AITER", section 1.2:
+ * the tensor is split into blocks of 32 elements, each with its own scale factor;
+ * section 1.1: MXFP8 = 8-bit elements plus a shared exponent).  Every row of x is cut
+ * into blocks of 32 consecutive elements; a block's scale is the power of two
+ * s = 2^e = 2^ceil(log2(amax / Fmax)), e >= -126 (the pages do not fix the exponent
+ * rule; this is the ue8m0 rule above, applied per block, so no element saturates),
+ * stored as the E8M0 byte e + 127; codes are q = saturate(RNE(x / s)).  Used for
+ * activations and, row by row, for weights alike.
+ *
+ *   x      bf16 [M][ldx] (first K columns); 16-byte aligned; ldx >= K, ldx % 8 == 0.
+ *   M, K   M >= 0, K > 0, K % 16 == 0 (a row's last block may hold 16 elements).
+ *   fmt    FP8_E4M3 or FP8_E5M2.
+ *   q      codes [M][K]; 16-byte aligned.
+ *   e8     exponent bytes in the tiled layout above, FP8_MX_SF_BYTES(M, K) bytes.
+ * Returns FP8_OK or an error status; M == 0 is a no-op.
+ */
+int fp8_mx_quant(const void* x, int64_t M, int64_t K, int64_t ldx, int fmt, void* q, void* e8,
+                 void* stream);
+
+/*
+ * fp8_mx_gemm -- FP8 GEMM with power-of-two scales per 32-element block of K, applied
+ * by the tensor core (the block-scaled MMA of sm_100a) to every product, accumulating
+ * all of K in fp32 with no per-K-block promotion:
+ *
+ *   y[m][n] = sum_k dec(qa[m][k]) 2^(ea(m, k/32) - 127) * dec(qw[n][k]) 2^(ew(n, k/32) - 127)
+ *
+ *   qa     E4M3 codes [M][K]; sfa its exponent bytes, tiled (FP8_MX_SF_BYTES(M, K)).
+ *   qw     E4M3 codes [N][K]; sfw its exponent bytes, tiled (FP8_MX_SF_BYTES(N, K)).
+ *   M >= 0, N > 0 with N % 16 == 0, K > 0 with K % 128 == 0; qa, qw, sfa, sfw, y
+ *   16-byte aligned.
+ *   out_dtype, y  as fp8_block_gemm.
+ * The ue8m0 block GEMM (act_quant / weight_quant with FP8_SCALE_UE8M0, fp8_block_gemm's
+ * scale layout) runs on this path after fp8_mx_pack_pow2 and gives fp8_block_gemm's
+ * result.  Accumulation: fp32 in tensor memory over all K (one rounding per 32-element
+ * block product); the tolerance this implies is stated with the parity tests.
+ */
+int fp8_mx_gemm(const void* qa, const void* sfa, const void* qw, const void* sfw, int64_t M, int64_t N,
+                int64_t K, int out_dtype, void* y, void* stream);
+
+/*
+ * fp8_mx_pack_pow2 -- converts fp32 power-of-two scales in fp8_block_gemm's layout
+ * (the ue8m0 scales of "FP8 推理提速 83.6%: DeepSeek-V3 在 AMD MI250 上的完整落地指南",
+ * 关键配置参数: scale_fmt ue8m0) into the tiled exponent layout of fp8_mx_gemm, each
+ * 128-element scale replicated onto its four 32-element blocks.
+ *
+ *   s          fp32 [rows][K/128] (row_block 1: act_quant's layout) or
+ *              fp32 [ceil(rows/128)][K/128] (row_block 128: weight_quant's 128x128 blocks).
+ *   rows, K    rows >= 0, K > 0 with K % 128 == 0.
+ *   sf         FP8_MX_SF_BYTES(rows, K) bytes; 16-byte aligned.
+ * A scale that is not a positive normal power of two is flagged: the next
+ * fp8_device_error() returns FP8_ERR_INVALID_SCALE.  rows == 0 is a no-op.
+ */
+int fp8_mx_pack_pow2(const float* s, int64_t rows, int64_t K, int row_block, void* sf, void* stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* fp8_status_string(int status);
 
@@ -136,7 +205,8 @@ const char* fp8_status_string(int status);
  * fp8_device_error -- synchronises `stream`, then reads and clears the
  * library's device-side error word on the current device.  Returns FP8_OK, or
  * FP8_ERR_TIMEOUT if a bounded wait in an earlier kernel ran out (that kernel
- * skipped its remaining work and returned), or FP8_ERR_CUDA.
+ * skipped its remaining work and returned), FP8_ERR_INVALID_SCALE if an earlier
+ * fp8_mx_pack_pow2 was given a scale that is not a power of two, or FP8_ERR_CUDA.
  */
 int fp8_device_error(void* stream);
 

@@ -74,3 +74,29 @@ def check_bf16(y_bits: np.ndarray, y_ref: np.ndarray, bound: np.ndarray, what: s
     assert n_allow <= ALLOWANCE_MAX_FRAC * d.size, \
         f"{what}: {n_allow} of {d.size} bf16 elements needed the cancellation allowance"
     return n_allow
+
+
+def untile_e8m0(buf, rows: int, K: int) -> np.ndarray:
+    """Tiled MXFP8 exponent bytes (the library's layout: 512-byte atoms of 128 rows x 4
+    blocks, byte (r % 32) * 16 + (r % 128 / 32) * 4 + j) -> row-major [rows, ceil(K/32)],
+    the oracle's layout.  A pure index permutation."""
+    b = buf.detach().cpu().numpy() if isinstance(buf, torch.Tensor) else np.asarray(buf)
+    nkb = (K + 127) // 128
+    nb = (K + 31) // 32
+    r = np.arange(rows)[:, None]
+    g = np.arange(nb)[None, :]
+    off = ((r >> 7) * nkb + (g >> 2)) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4 + (g & 3)
+    return b[off]
+
+
+def tile_e8m0(rm: np.ndarray, rows: int, K: int) -> np.ndarray:
+    """Row-major [rows, K/32] exponent bytes -> the library's tiled layout (inverse of
+    untile_e8m0; bytes of padding rows are 0)."""
+    nkb = (K + 127) // 128
+    out = np.zeros(((rows + 127) // 128) * nkb * 512, np.uint8)
+    nb = rm.shape[1]
+    r = np.arange(rows)[:, None]
+    g = np.arange(nb)[None, :]
+    off = ((r >> 7) * nkb + (g >> 2)) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4 + (g & 3)
+    out[off] = rm
+    return out

@@ -12,7 +12,7 @@ import fp8_block_scaled_12_b200 as F
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "fp8lin.h")
 
-OK, INVALID, SHAPE, ALIGN, UNSUP, CUDA, TIMEOUT = range(7)
+OK, INVALID, SHAPE, ALIGN, UNSUP, CUDA, TIMEOUT, BADSCALE = range(8)
 FAKE = 0x7F0000000000       # 16-byte aligned, never dereferenced
 S = None                    # default stream
 
@@ -37,7 +37,7 @@ def test_library_exports_every_declared_function():
 
 def test_status_strings():
     assert F.fp8_status_string(OK) == "ok"
-    for c in range(1, 7):
+    for c in range(1, 8):
         assert F.fp8_status_string(c) not in ("ok", "unknown status")
     assert F.fp8_status_string(99) == "unknown status"
 
@@ -134,3 +134,44 @@ def test_python_binding_refuses_stacked_weights():
     w = torch.zeros(2, 200, 256, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         F.fp8_weight_quant(w, torch.zeros(2, 200, 256, dtype=torch.uint8), torch.zeros(4, 2))
+
+
+def test_mx_validation():
+    mq = F.lib.fp8_mx_quant
+    # (x, M, K, ldx, fmt, q, e8, stream)
+    assert mq(FAKE, -1, 64, 64, 0, FAKE, FAKE, S) == INVALID
+    assert mq(FAKE, 4, 64, 32, 0, FAKE, FAKE, S) == INVALID                # ldx < K
+    assert mq(FAKE, 4, 64, 64, 3, FAKE, FAKE, S) == INVALID                # bad format
+    assert mq(FAKE, 4, 72, 72, 0, FAKE, FAKE, S) == SHAPE                  # K % 16
+    assert mq(FAKE, 4, 64, 64, 0, FAKE, None, S) == INVALID
+    assert mq(FAKE + 8, 4, 64, 64, 0, FAKE, FAKE, S) == ALIGN
+    assert mq(FAKE, 0, 64, 64, 0, None, None, S) == OK
+    mg = F.lib.fp8_mx_gemm
+    # (qa, sfa, qw, sfw, M, N, K, out, y, stream)
+    assert mg(FAKE, FAKE, FAKE, FAKE, 16, 256, 192, 0, FAKE, S) == SHAPE    # K % 128
+    assert mg(FAKE, FAKE, FAKE, FAKE, 16, 120, 256, 0, FAKE, S) == SHAPE    # N % 16
+    assert mg(FAKE, FAKE, FAKE, FAKE, 16, 256, 256, 3, FAKE, S) == INVALID  # out dtype
+    assert mg(FAKE, FAKE + 4, FAKE, FAKE, 16, 256, 256, 0, FAKE, S) == ALIGN  # scales: 16-byte bulk copies
+    assert mg(FAKE, FAKE, FAKE, FAKE, 0, 256, 256, 0, None, S) == OK         # M == 0
+    mp = F.lib.fp8_mx_pack_pow2
+    # (s, rows, K, row_block, sf, stream)
+    assert mp(FAKE, 16, 256, 64, FAKE, S) == INVALID                         # row block
+    assert mp(FAKE, 16, 200, 1, FAKE, S) == SHAPE                            # K % 128
+    assert mp(FAKE, 16, 256, 1, FAKE + 8, S) == ALIGN
+    assert mp(FAKE, 0, 256, 128, None, S) == OK
+
+
+def test_python_binding_checks_mx_operands():
+    import torch
+    M, N, K = 4, 256, 256
+    qa = torch.zeros(M, K, dtype=torch.uint8)
+    qw = torch.zeros(N, K, dtype=torch.uint8)
+    y = torch.zeros(M, N, dtype=torch.bfloat16)
+    assert F.mx_sf_bytes(M, K) == 1024 and F.mx_sf_bytes(129, 128) == 1024 and F.mx_sf_bytes(1, 16) == 512
+    with pytest.raises(ValueError):      # row-major [M, K/32] bytes are not the tiled layout
+        F.fp8_mx_gemm(qa, torch.zeros(M, K // 32, dtype=torch.uint8), qw,
+                      torch.zeros(F.mx_sf_bytes(N, K), dtype=torch.uint8), y)
+    with pytest.raises(TypeError):
+        F.fp8_mx_gemm(qa, torch.zeros(F.mx_sf_bytes(M, K)), qw, torch.zeros(F.mx_sf_bytes(N, K)), y)
+    with pytest.raises(ValueError):      # weight scales per 128 x 128 block
+        F.fp8_mx_pack_pow2(torch.zeros(N, K // 128), N, K, 128, torch.zeros(F.mx_sf_bytes(N, K), dtype=torch.uint8))
