@@ -365,6 +365,15 @@ def measure_rows(dev, peaks):
         b = M * K * 3 + 4
         res[name + " 16384x7168"] = {"GB/s (algorithmic 3 B/elt)": round(b / ms / 1e6, 1),
                                       "frac_hbm": round(b / ms / 1e6 / hbm, 4)}
+    # delayed scaling: one pass, previous step's scale, amax history of 16 (3 B/elt + state)
+    ds = F.DelayedScaling(hist_len=16, device=dev)
+    nclip = torch.empty(1, dtype=torch.int64, device=dev)
+    sused = torch.empty(1, dtype=torch.float32, device=dev)
+    ms = time_launches(lambda: F.fp8_delayed_quant(x, q, ds.scale, ds.pos, ds.history, nclip, sused), 20)
+    b = M * K * 3
+    res["delayed_scaling e4m3 16384x7168 (single pass)"] = {"GB/s (3 B/elt)": round(b / ms / 1e6, 1),
+                                                            "frac_hbm": round(b / ms / 1e6 / hbm, 4),
+                                                            "us": round(ms * 1e3, 2)}
     del x, q, s
     # weight_quant 128x128 on the prefill weight
     w = synth.weights(28672, 8192, 0.02, seed=0, device=dev)
@@ -505,7 +514,7 @@ def cpu_baseline_prefill(S, dev):
     usable, reported = host_cores()
     qw = S["qw"].cpu().numpy()
     sw = S["sw"].cpu().numpy()
-    rows_mt = 4 * usable                  # about 4 s of work on every core
+    rows_mt = 16 * usable                 # about 10 s of work on every core
     x = S["x"][:rows_mt].cpu()
     qa, sa = O.act_quant(x)
 

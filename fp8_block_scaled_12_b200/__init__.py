@@ -21,7 +21,8 @@ import torch
 __all__ = [
     "E4M3", "E5M2", "SCALE_FP32", "SCALE_UE8M0", "OUT_BF16", "OUT_FP32", "Fp8Error", "LIB_PATH",
     "fp8_act_quant", "fp8_weight_quant", "fp8_block_gemm", "fp8_grouped_gemm", "fp8_mx_quant", "fp8_mx_gemm",
-    "fp8_mx_pack_pow2", "fp8_status_string", "fp8_device_error", "fp8_selftest_bounded_wait",
+    "fp8_mx_pack_pow2", "fp8_delayed_quant", "DelayedScaling", "AMAX_MOST_RECENT", "AMAX_MAX",
+    "fp8_status_string", "fp8_device_error", "fp8_selftest_bounded_wait",
     "act_quant", "weight_quant", "block_gemm", "grouped_gemm", "mx_quant", "mx_gemm", "mx_pack_pow2",
     "mx_sf_bytes", "EXPORTS",
 ]
@@ -30,12 +31,14 @@ E4M3, E5M2 = 0, 1
 SCALE_FP32, SCALE_UE8M0 = 0, 1
 OUT_BF16, OUT_FP32 = 0, 1
 MX_BLOCK = 32
+AMAX_MOST_RECENT, AMAX_MAX = 0, 1
 FP8_OK = 0
 FP8_ERR_INVALID_SCALE = 7
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfp8lin.so")
 EXPORTS = ("fp8_act_quant", "fp8_weight_quant", "fp8_block_gemm", "fp8_grouped_gemm", "fp8_mx_quant",
-           "fp8_mx_gemm", "fp8_mx_pack_pow2", "fp8_status_string", "fp8_device_error", "fp8_selftest_bounded_wait")
+           "fp8_mx_gemm", "fp8_mx_pack_pow2", "fp8_delayed_quant", "fp8_status_string", "fp8_device_error",
+           "fp8_selftest_bounded_wait")
 
 
 class Fp8Error(RuntimeError):
@@ -56,12 +59,14 @@ def _load() -> ctypes.CDLL:
     L.fp8_mx_quant.argtypes = [vp, i64, i64, i64, ci, vp, vp, vp]
     L.fp8_mx_gemm.argtypes = [vp, vp, vp, vp, i64, i64, i64, ci, vp, vp]
     L.fp8_mx_pack_pow2.argtypes = [vp, i64, i64, ci, vp, vp]
+    L.fp8_delayed_quant.argtypes = [vp, i64, ci, ctypes.c_float, i64, ci, vp, vp, vp, vp, vp, vp, vp]
     L.fp8_status_string.argtypes = [ci]
     L.fp8_status_string.restype = ctypes.c_char_p
     L.fp8_device_error.argtypes = [vp]
     L.fp8_selftest_bounded_wait.argtypes = [i64, vp]
     for name in ("fp8_act_quant", "fp8_weight_quant", "fp8_block_gemm", "fp8_grouped_gemm", "fp8_mx_quant",
-                 "fp8_mx_gemm", "fp8_mx_pack_pow2", "fp8_device_error", "fp8_selftest_bounded_wait"):
+                 "fp8_mx_gemm", "fp8_mx_pack_pow2", "fp8_delayed_quant", "fp8_device_error",
+                 "fp8_selftest_bounded_wait"):
         getattr(L, name).restype = ci
     return L
 
@@ -233,6 +238,45 @@ def fp8_mx_pack_pow2(s: torch.Tensor, rows: int, K: int, row_block: int, sf: tor
     _expect(s, (rows if row_block == 1 else (rows + 127) // 128, K // 128), "s")
     _expect(sf, (mx_sf_bytes(rows, K),), "sf", torch.uint8)
     _check("fp8_mx_pack_pow2", lib.fp8_mx_pack_pow2(_ptr(s), rows, K, row_block, _ptr(sf), _stream(stream)))
+
+
+def fp8_delayed_quant(x: torch.Tensor, q: torch.Tensor, scale: torch.Tensor, pos: torch.Tensor,
+                      history: torch.Tensor, n_clipped: torch.Tensor, s_used: torch.Tensor, fmt: int = E4M3,
+                      target: float = 400.0, algo: int = AMAX_MAX, stream=None) -> None:
+    """One delayed-scaling step over all elements of bf16 x (any shape, contiguous)."""
+    for t in (x, q, scale, pos, history, n_clipped, s_used):
+        assert t.is_contiguous()
+    assert x.dtype == torch.bfloat16 and q.numel() == x.numel()
+    _expect(scale, (1,), "scale", torch.float32)
+    _expect(pos, (1,), "pos", torch.int32)
+    assert history.dtype == torch.float32 and history.dim() == 1
+    _expect(n_clipped, (1,), "n_clipped", torch.int64)
+    _expect(s_used, (1,), "s_used", torch.float32)
+    _check("fp8_delayed_quant", lib.fp8_delayed_quant(_ptr(x), x.numel(), fmt, float(target), history.numel(),
+                                                      algo, _ptr(scale), _ptr(pos), _ptr(history), _ptr(_u8(q)),
+                                                      _ptr(n_clipped), _ptr(s_used), _stream(stream)))
+
+
+class DelayedScaling:
+    """Device state of delayed per-tensor scaling (initial scale 1.0, empty history),
+    stepped with fp8_delayed_quant; `step(x)` returns (codes, scale used, clipped count
+    as a device tensor)."""
+
+    def __init__(self, hist_len: int = 16, fmt: int = E4M3, target: float | None = None,
+                 algo: int = AMAX_MAX, device="cuda"):
+        self.fmt, self.algo = fmt, algo
+        self.target = target if target is not None else (400.0 if fmt == E4M3 else 57344.0 * 400.0 / 448.0)
+        self.scale = torch.ones(1, dtype=torch.float32, device=device)
+        self.pos = torch.zeros(1, dtype=torch.int32, device=device)
+        self.history = torch.zeros(hist_len, dtype=torch.float32, device=device)
+
+    def step(self, x: torch.Tensor, stream=None):
+        q = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+        n_clipped = torch.empty(1, dtype=torch.int64, device=x.device)
+        s_used = torch.empty(1, dtype=torch.float32, device=x.device)
+        fp8_delayed_quant(x, q, self.scale, self.pos, self.history, n_clipped, s_used, self.fmt, self.target,
+                          self.algo, stream)
+        return q, s_used, n_clipped
 
 
 def fp8_device_error(stream=None) -> int:

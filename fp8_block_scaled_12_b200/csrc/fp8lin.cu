@@ -324,6 +324,35 @@ int fp8_grouped_gemm(const void* qa, const float* sa, const void* qw, const floa
   return launch_swap<160, 3, 5, 28>(qa, qw, a, E * N, static_cast<cudaStream_t>(stream));
 }
 
+int fp8_delayed_quant(const void* x, int64_t n, int fmt, float target, int64_t hist_len, int algo, float* scale,
+                      int32_t* pos, float* history, void* q, uint64_t* n_clipped, float* s_used, void* stream) {
+  if (n < 0 || hist_len < 1 || hist_len > 65536) return FP8_ERR_INVALID_ARG;
+  if (fmt != FP8_E4M3 && fmt != FP8_E5M2) return FP8_ERR_INVALID_ARG;
+  if (algo != FP8_AMAX_MOST_RECENT && algo != FP8_AMAX_MAX) return FP8_ERR_INVALID_ARG;
+  if (!(target > 0.0f) || !(target < 3.0e38f)) return FP8_ERR_INVALID_ARG;
+  if (!scale || !pos || !history || !n_clipped || !s_used || (n > 0 && (!x || !q))) return FP8_ERR_INVALID_ARG;
+  if (n % 8 != 0) return FP8_ERR_SHAPE;
+  if ((n > 0 && (!aligned(x, 16) || !aligned(q, 16))) || !aligned(scale, 4) || !aligned(pos, 4) ||
+      !aligned(history, 4) || !aligned(n_clipped, 8) || !aligned(s_used, 4))
+    return FP8_ERR_ALIGNMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(n_clipped, 0, sizeof(uint64_t), st) != cudaSuccess) return FP8_ERR_CUDA;
+  const int64_t n8 = n / 8;
+  int64_t blocks = (n8 + 255) / 256;
+  const int64_t cap = int64_t(num_sms()) * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  const uint16_t* xb = static_cast<const uint16_t*>(x);
+  uint8_t* qb = static_cast<uint8_t*>(q);
+  unsigned long long* nc = reinterpret_cast<unsigned long long*>(n_clipped);
+  if (fmt == FP8_E4M3)
+    k_delayed_cast<kE4M3><<<int(blocks), 256, 0, st>>>(xb, n8, scale, pos, int(hist_len), history, qb, nc, s_used);
+  else
+    k_delayed_cast<kE5M2><<<int(blocks), 256, 0, st>>>(xb, n8, scale, pos, int(hist_len), history, qb, nc, s_used);
+  k_delayed_finalize<<<1, 32, 0, st>>>(target, int(hist_len), algo, scale, pos, history);
+  return cuda_status(cudaGetLastError());
+}
+
 int fp8_mx_quant(const void* x, int64_t M, int64_t K, int64_t ldx, int fmt, void* q, void* e8, void* stream) {
   if (M < 0 || K <= 0 || ldx < K) return FP8_ERR_INVALID_ARG;
   if (fmt != FP8_E4M3 && fmt != FP8_E5M2) return FP8_ERR_INVALID_ARG;

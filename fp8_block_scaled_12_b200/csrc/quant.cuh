@@ -326,4 +326,131 @@ __global__ void k_tensor_scale(unsigned int* slot) {
   *reinterpret_cast<float*>(slot) = sc.s;
 }
 
+// ------------------------------------------------------- delayed scaling
+// One step of delayed per-tensor scaling ("ROCm 7 ... AITER", section 4.3: divide by the
+// previous step's scale, clamp to +-Fmax, cast; the next scale comes from this step's
+// amax; section 6: an amax history whose max sets the scale; the checklist's count of
+// clipped elements).  One pass over x: k_delayed_cast casts with the stored scale,
+// folds the tensor's amax into the history slot of this step (integer atomicMax on
+// the bits of non-negative floats) and counts the elements whose quotient lies beyond
+// +-Fmax; k_delayed_finalize turns the history into the next step's scale.
+
+// x / s for an arbitrary positive normal fp32 scale s (the previous step's scale):
+// Markstein's correction on a correctly rounded reciprocal as in GroupScale, with s
+// brought into [2^-64, 2^64) by an exact power of two so the reciprocal stays normal,
+// and quotients already beyond 2^100 (which saturate whatever their last bits) taken
+// as they are, so an overflowing quotient never turns into NaN.  tests/
+// division_delayed.c checks, for every bf16 x and scales of every binary exponent, that
+// the FP8 code and the clipped flag |q| > Fmax equal those of the IEEE quotient.
+struct DelayedDiv {
+  float pre, ss, r;
+  __device__ __forceinline__ explicit DelayedDiv(float s) {
+    pre = (s < 5.42101086242752217004e-20f) ? 18446744073709551616.0f
+          : (s >= 18446744073709551616.0f ? 5.42101086242752217004e-20f : 1.0f);   // 2^64 / 2^-64 / 1
+    ss = __fmul_rn(s, pre);
+    r = __frcp_rn(ss);
+  }
+  __device__ __forceinline__ float apply(float x) const {
+    const float xs = __fmul_rn(x, pre);
+    const float q0 = __fmul_rn(xs, r);
+    if (fabsf(q0) >= 1.2676506002282294e30f) return q0;                              // 2^100
+    return copysignf(__fmaf_rn(__fmaf_rn(-q0, ss, xs), r, q0), x);
+  }
+};
+
+template <int FMT>
+__device__ __forceinline__ uint2 delayed8(const uint4 v, const DelayedDiv& dv, uint32_t& clipped) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t c[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float lo = dv.apply(bf16_lo(w[i])), hi = dv.apply(bf16_hi(w[i]));
+    clipped += (fabsf(lo) > FmtTraits<FMT>::kMax ? 1u : 0u) + (fabsf(hi) > FmtTraits<FMT>::kMax ? 1u : 0u);
+    c[i] = cvt2<FMT>(lo, hi);
+  }
+  return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+}
+
+// The caller owns the slot index; it is taken modulo the history length so a corrupted
+// state can never address outside the history.
+__device__ __forceinline__ int delayed_slot(const int32_t* pos, int hist_len) {
+  return ((*pos % hist_len) + hist_len) % hist_len;
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(256) k_delayed_cast(const uint16_t* __restrict__ x, int64_t n8,
+                                                      const float* __restrict__ scale,
+                                                      const int32_t* __restrict__ pos, int hist_len, float* history,
+                                                      uint8_t* __restrict__ q, unsigned long long* n_clipped,
+                                                      float* s_used) {
+  __shared__ float red_a[8];
+  __shared__ uint32_t red_c[8];
+  const float s = *scale;
+  const DelayedDiv dv(s);
+  const uint4* p = reinterpret_cast<const uint4*>(x);
+  uint2* o = reinterpret_cast<uint2*>(q);
+  float a = 0.0f;
+  uint32_t clipped = 0;
+  const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+  int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  for (; i + 3 * stride < n8; i += 4 * stride) {        // four 16-byte loads in flight
+    uint4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) v[u] = ldg_stream(p + i + u * stride);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      a = amax8(v[u], a);
+      o[i + u * stride] = delayed8<FMT>(v[u], dv, clipped);
+    }
+  }
+  for (; i < n8; i += stride) {
+    const uint4 v = ldg_stream(p + i);
+    a = amax8(v, a);
+    o[i] = delayed8<FMT>(v, dv, clipped);
+  }
+#pragma unroll
+  for (int d = 16; d > 0; d >>= 1) {
+    a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, d));
+    clipped += __shfl_xor_sync(0xffffffffu, clipped, d);
+  }
+  if ((threadIdx.x & 31) == 0) {
+    red_a[threadIdx.x >> 5] = a;
+    red_c[threadIdx.x >> 5] = clipped;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint64_t c = 0;
+    for (int w = 0; w < 8; ++w) {
+      a = fmaxf(a, red_a[w]);
+      c += red_c[w];
+    }
+    atomicMax(reinterpret_cast<unsigned int*>(history + delayed_slot(pos, hist_len)), __float_as_uint(a));
+    if (c) atomicAdd(n_clipped, (unsigned long long)c);
+    if (blockIdx.x == 0) *s_used = s;
+  }
+}
+
+// One warp: next scale = (max over the history, or this step's amax) / target, at
+// least 2^-126; then clear the next slot and advance the slot index.
+__global__ void k_delayed_finalize(float target, int hist_len, int algo, float* scale, int32_t* pos,
+                                   float* history) {
+  const int lane = threadIdx.x;
+  const int p = delayed_slot(pos, hist_len);
+  float a = 0.0f;
+  if (algo == 1) {
+    for (int h = lane; h < hist_len; h += 32) a = fmaxf(a, history[h]);
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, d));
+  } else {
+    a = history[p];
+  }
+  __syncwarp();
+  if (lane == 0) {
+    *scale = fmaxf(__fdiv_rn(a, target), 1.17549435082228750797e-38f);   // 2^-126
+    const int np = (p + 1) % hist_len;
+    history[np] = 0.0f;
+    *pos = np;
+  }
+}
+
 }  // namespace fp8lin

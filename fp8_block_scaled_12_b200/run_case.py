@@ -45,7 +45,7 @@ def timed(fn, warm, iters):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--op", required=True, choices=["act_quant", "weight_quant", "gemm", "grouped", "mx_quant",
-                                                    "mx_gemm"])
+                                                    "mx_gemm", "delayed"])
     ap.add_argument("--M", type=int, default=4096)
     ap.add_argument("--N", type=int, default=28672)
     ap.add_argument("--K", type=int, default=8192)
@@ -94,6 +94,16 @@ def main():
         b = qa.numel() + qw.numel() + y.numel() * y.element_size() + sa.numel() * 4 + sw.numel() * 4
         print(f"gemm M={a.M} N={a.N} K={a.K} {a.scale} {a.out}: {ms * 1e3:.2f} us  {fl / ms / 1e9:.1f} TFLOPS  "
               f"{b / ms / 1e6:.1f} GB/s")
+    elif a.op == "delayed":
+        x = synth.activations(a.M, a.K, seed=0, dist=a.dist, device=dev)
+        q = torch.empty((a.M, a.K), dtype=torch.uint8, device=dev)
+        ds = F.DelayedScaling(hist_len=16, fmt=fmt, device=dev)
+        nclip = torch.empty(1, dtype=torch.int64, device=dev)
+        sused = torch.empty(1, dtype=torch.float32, device=dev)
+        ms = timed(lambda: F.fp8_delayed_quant(x, q, ds.scale, ds.pos, ds.history, nclip, sused, fmt=fmt,
+                                               target=ds.target), a.warm, a.iters)
+        b = a.M * a.K * 3
+        print(f"delayed M={a.M} K={a.K} {a.fmt}: {ms * 1e3:.2f} us  {b / ms / 1e6:.1f} GB/s (3 B/elt)")
     elif a.op == "mx_quant":
         x = synth.activations(a.M, a.K, seed=0, dist=a.dist, device=dev)
         q = torch.empty((a.M, a.K), dtype=torch.uint8, device=dev)

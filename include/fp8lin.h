@@ -198,6 +198,36 @@ int fp8_mx_gemm(const void* qa, const void* sfa, const void* qw, const void* sfw
  */
 int fp8_mx_pack_pow2(const float* s, int64_t rows, int64_t K, int row_block, void* sf, void* stream);
 
+/* History rule of fp8_delayed_quant. */
+typedef enum { FP8_AMAX_MOST_RECENT = 0, FP8_AMAX_MAX = 1 } fp8_amax_algo;
+
+/*
+ * fp8_delayed_quant -- one step of delayed per-tensor scaling, a single pass over x
+ * ("ROCm 7 原生 FP8/MXFP8 ... AITER", section 4.3 延迟缩放: the tensor is divided by the
+ * scale of the PREVIOUS step, clamped to +-Fmax and cast; the scale of the next step is
+ * derived from this step's amax with a margin, amax / 400 for E4M3, starting from 1.0;
+ * section 6: an amax history, "max" over it; its checklist tracks the share of clipped
+ * elements):
+ *   q[i]        = saturate(RNE(x[i] / s_prev)),  s_prev = *scale on entry
+ *   *n_clipped  = number of i with |fl32(x[i] / s_prev)| > Fmax
+ *   *s_used     = s_prev (dequantise with x ~= dec(q) * s_used)
+ *   history[*pos] = max |x|;  then  *scale = max(A / target, 2^-126) with A = the max
+ *   over history[0..hist_len) (FP8_AMAX_MAX) or this step's amax (FP8_AMAX_MOST_RECENT);
+ *   history[(*pos + 1) % hist_len] = 0;  *pos = (*pos + 1) % hist_len.
+ *
+ *   x        bf16 [n], 16-byte aligned; n >= 0, n % 8 == 0.
+ *   fmt      FP8_E4M3 or FP8_E5M2; target > 0, finite (the page: 400 for E4M3).
+ *   scale, pos, history   DEVICE state owned by the caller and carried from step to
+ *            step: fp32 [1], int32 [1], fp32 [hist_len] (1 <= hist_len <= 65536).
+ *            Before the first step: *scale = 1.0, *pos = 0, history all 0.  Steps on
+ *            one state must be ordered on one stream.
+ *   q        codes [n], 16-byte aligned.
+ *   n_clipped  DEVICE uint64 [1] (8-byte aligned); s_used DEVICE fp32 [1].
+ * Returns FP8_OK or an error status.  Enqueues a memset of *n_clipped and two kernels.
+ */
+int fp8_delayed_quant(const void* x, int64_t n, int fmt, float target, int64_t hist_len, int algo, float* scale,
+                      int32_t* pos, float* history, void* q, uint64_t* n_clipped, float* s_used, void* stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* fp8_status_string(int status);
 

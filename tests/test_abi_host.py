@@ -52,7 +52,7 @@ def test_act_quant_validation():
     assert aq(FAKE, 4, 128, 64, 128, 0, 0, FAKE, FAKE, S) == INVALID        # ldx < K
     assert aq(FAKE, 4, 128, 128, 128, 2, 0, FAKE, FAKE, S) == INVALID       # bad format
     assert aq(FAKE, 4, 128, 128, 128, 0, 7, FAKE, FAKE, S) == INVALID       # bad scale format
-    assert aq(FAKE, 4, 128, 128, 32, 0, 0, FAKE, FAKE, S) == UNSUP          # group 32 not built
+    assert aq(FAKE, 4, 128, 128, 32, 0, 0, FAKE, FAKE, S) == UNSUP          # 32-element blocks: fp8_mx_quant
     assert aq(FAKE, 4, 136, 136, 128, 0, 0, FAKE, FAKE, S) == SHAPE         # K % 16
     assert aq(None, 4, 128, 128, 128, 0, 0, FAKE, FAKE, S) == INVALID       # null x
     assert aq(FAKE + 8, 4, 128, 128, 128, 0, 0, FAKE, FAKE, S) == ALIGN     # x not 16-byte aligned
@@ -175,3 +175,18 @@ def test_python_binding_checks_mx_operands():
         F.fp8_mx_gemm(qa, torch.zeros(F.mx_sf_bytes(M, K)), qw, torch.zeros(F.mx_sf_bytes(N, K)), y)
     with pytest.raises(ValueError):      # weight scales per 128 x 128 block
         F.fp8_mx_pack_pow2(torch.zeros(N, K // 128), N, K, 128, torch.zeros(F.mx_sf_bytes(N, K), dtype=torch.uint8))
+
+
+def test_delayed_quant_validation():
+    dq = F.lib.fp8_delayed_quant
+    F32 = ctypes.c_float
+    # (x, n, fmt, target, hist_len, algo, scale, pos, history, q, n_clipped, s_used, stream)
+    assert dq(FAKE, -8, 0, F32(400.0), 16, 1, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, S) == INVALID
+    assert dq(FAKE, 64, 0, F32(400.0), 0, 1, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, S) == INVALID    # history length
+    assert dq(FAKE, 64, 0, F32(0.0), 16, 1, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, S) == INVALID     # target
+    assert dq(FAKE, 64, 0, F32(400.0), 16, 2, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, S) == INVALID   # algo
+    assert dq(FAKE, 64, 5, F32(400.0), 16, 1, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, S) == INVALID   # format
+    assert dq(FAKE, 64, 0, F32(400.0), 16, 1, None, FAKE, FAKE, FAKE, FAKE, FAKE, S) == INVALID   # state
+    assert dq(FAKE, 60, 0, F32(400.0), 16, 1, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, S) == SHAPE     # n % 8
+    assert dq(FAKE + 8, 64, 0, F32(400.0), 16, 1, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, S) == ALIGN
+    assert dq(FAKE, 64, 0, F32(400.0), 16, 1, FAKE, FAKE, FAKE, FAKE, FAKE + 4, FAKE, S) == ALIGN  # uint64 count

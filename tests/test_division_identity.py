@@ -27,3 +27,16 @@ def test_fast_division_gives_ieee_codes(checker):
     r = subprocess.run([checker, stride], capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stdout + r.stderr
     assert "code_mismatches=0" in r.stdout
+
+
+def test_delayed_scaling_division_gives_ieee_codes_and_clip_flags(tmp_path):
+    """The delayed-scaling kernel divides by an arbitrary previous-step scale: for every
+    bf16 x and scales of every binary exponent (8 significands each), its quotient must
+    give the IEEE quotient's FP8 code and the same clipped flag (tests/division_delayed.c)."""
+    exe = str(tmp_path / "division_delayed")
+    subprocess.check_call(["gcc", "-O2", "-ffp-contract=off", "-fno-fast-math", "-o", exe,
+                           os.path.join(HERE, "division_delayed.c"),
+                           os.path.join(ROOT, "oracle", "fp8_oracle.c"), "-lm", "-lpthread"])
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert r.stdout.count("code_mismatches=0 clip_mismatches=0") == 2
