@@ -59,6 +59,8 @@ def lib():
         L.orc_mx_quant.argtypes = [vp, i64, i64, i64, i64, ctypes.c_int, vp, vp]
         L.orc_mx_gemm_rows.restype = None
         L.orc_mx_gemm_rows.argtypes = [vp, vp, vp, vp, i64, i64, vp, i64, vp, vp]
+        L.orc_weight_dequant.restype = None
+        L.orc_weight_dequant.argtypes = [vp, vp, i64, i64, i64, ctypes.c_int, vp]
         L.orc_delayed_quant.restype = None
         L.orc_delayed_quant.argtypes = [vp, i64, ctypes.c_int, ctypes.c_float, i64, ctypes.c_int, vp, vp, vp, vp,
                                         vp, vp]
@@ -312,3 +314,19 @@ def delayed_quant(x, state: DelayedScalingState, fmt: int = E4M3, target: float 
     lib().orc_delayed_quant(_ptr(xb), xb.size, fmt, float(target), state.history.size, algo, _ptr(state.scale),
                             _ptr(state.pos), _ptr(state.history), _ptr(q), _ptr(n_clip), _ptr(s_used))
     return q, int(n_clip[0]), float(s_used[0])
+
+
+def weight_dequant(q, s_inv, block: int = 128, fmt: int = E4M3, threads: int = 1):
+    """FP8 codes [N, K] + scales -> bf16 bit patterns [N, K] (fp32 product, one RNE to bf16)."""
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    s_inv = np.ascontiguousarray(s_inv, dtype=np.float32)
+    N, K = q.shape
+    out = np.empty((N, K), dtype=np.uint16)
+    nbk = (K + block - 1) // block if block else 1
+
+    def part(r0, r1):
+        sp = _ptr(s_inv) + ((r0 // block) * nbk * 4 if block else 0)
+        lib().orc_weight_dequant(_ptr(q) + r0 * K, sp, r1 - r0, K, block, fmt, _ptr(out) + r0 * K * 2)
+
+    _run_parallel(part, _split(N, threads, block if block else 1), threads)
+    return out

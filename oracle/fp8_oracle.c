@@ -426,3 +426,24 @@ void orc_delayed_quant(const uint16_t *x, int64_t n, int fmt, float target, int6
     history[p] = 0.0f;
     *pos = p;
 }
+
+/* ------------------------------------------------------ weight dequantisation */
+
+/* The BF16 path of the DeepSeek-V3 page ([P4] 运行时: weight = weight_dequant(weight,
+ * weight.scale), then a plain GEMM; FP8 权重转换: fp8_cast_bf16.py turns the FP8
+ * checkpoint into BF16): w[n][k] = dec(q[n][k]) * s_inv[n/block][k/block] formed as one
+ * IEEE fp32 product (the reading taken: the codes are widened to fp32 and multiplied
+ * by the fp32 scale, as a GEMM input would be), then rounded to bf16 to nearest even.
+ * block == 0 uses the single per-tensor scale s_inv[0].  out holds bf16 bit patterns. */
+void orc_weight_dequant(const uint8_t *q, const float *s_inv, int64_t N, int64_t K, int64_t block,
+                        int fmt, uint16_t *out)
+{
+    int64_t nbk = block > 0 ? (K + block - 1) / block : 1;
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t k = 0; k < K; ++k) {
+            float s = block > 0 ? s_inv[(n / block) * nbk + k / block] : s_inv[0];
+            float v = (float)orc_decode(q[n * K + k], fmt) * s;     /* one fp32 rounding */
+            out[n * K + k] = orc_round_bf16((double)v);             /* exact widening, one bf16 rounding */
+        }
+    }
+}
