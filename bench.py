@@ -419,7 +419,43 @@ def measure_rows(dev, peaks):
                                                     "frac_hbm": round(b / ms / 1e6 / hbm, 4)}
     assert F.fp8_device_error() == 0
     del qwe, swe, qa, sa, y
+    res.update(measure_fused_rows(dev, peaks))
     res.update(measure_mx_rows(dev, peaks))
+    return res
+
+
+def measure_fused_rows(dev, peaks):
+    """Steps beside the GEMM: the BF16 path's weight dequantisation, and the prefill GEMM
+    whose epilogue quantises its output for the next layer (no separate act_quant pass)."""
+    import torch
+    import fp8_block_scaled_12_b200 as F
+    import synth
+    res = {}
+    hbm = peaks["hbm_gbs"]
+    fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
+    p = synth.PREFILL.params
+    M, N, K = p["M"], p["N"], p["K"]
+    w = synth.weights(N, K, p["w_std"], seed=0, device=dev)
+    qw, sw = F.weight_quant(w)
+    wb = torch.empty_like(w)
+    ms = time_launches(lambda: F.fp8_weight_dequant(qw, sw, wb), 10)
+    b = N * K * 3 + sw.numel() * 4
+    res["weight_dequant 28672x8192"] = {"GB/s": round(b / ms / 1e6, 1), "frac_hbm": round(b / ms / 1e6 / hbm, 4),
+                                        "us": round(ms * 1e3, 1)}
+    del w, wb
+    x = synth.activations(M, K, seed=0, device=dev)
+    qa, sa = F.act_quant(x)
+    qy = torch.empty((M, N), dtype=torch.uint8, device=dev)
+    sy = torch.empty((M, N // 128), dtype=torch.float32, device=dev)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    fl = 2.0 * M * N * K
+    ms = time_launches(lambda: F.fp8_block_gemm_quant(qa, sa, qw, sw, qy, sy), 10)
+    res["block_gemm_quant prefill 4096x28672x8192 (codes + scales out, no y)"] = {
+        "us": round(ms * 1e3, 1), "TFLOPS": round(fl / ms / 1e9, 1), "frac_fp8_peak": round(fl / ms / 1e9 / fp8_peak, 4)}
+    ms = time_launches(lambda: F.fp8_block_gemm_quant(qa, sa, qw, sw, qy, sy, y), 10)
+    res["block_gemm_quant prefill 4096x28672x8192 (y, codes and scales out)"] = {
+        "us": round(ms * 1e3, 1), "TFLOPS": round(fl / ms / 1e9, 1), "frac_fp8_peak": round(fl / ms / 1e9 / fp8_peak, 4)}
+    assert F.fp8_device_error() == 0
     return res
 
 

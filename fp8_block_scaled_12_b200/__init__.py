@@ -22,6 +22,7 @@ __all__ = [
     "E4M3", "E5M2", "SCALE_FP32", "SCALE_UE8M0", "OUT_BF16", "OUT_FP32", "Fp8Error", "LIB_PATH",
     "fp8_act_quant", "fp8_weight_quant", "fp8_block_gemm", "fp8_grouped_gemm", "fp8_mx_quant", "fp8_mx_gemm",
     "fp8_mx_pack_pow2", "fp8_delayed_quant", "DelayedScaling", "AMAX_MOST_RECENT", "AMAX_MAX",
+    "fp8_block_gemm_quant", "fp8_weight_dequant", "block_gemm_quant", "weight_dequant",
     "fp8_status_string", "fp8_device_error", "fp8_selftest_bounded_wait",
     "act_quant", "weight_quant", "block_gemm", "grouped_gemm", "mx_quant", "mx_gemm", "mx_pack_pow2",
     "mx_sf_bytes", "EXPORTS",
@@ -37,8 +38,8 @@ FP8_ERR_INVALID_SCALE = 7
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfp8lin.so")
 EXPORTS = ("fp8_act_quant", "fp8_weight_quant", "fp8_block_gemm", "fp8_grouped_gemm", "fp8_mx_quant",
-           "fp8_mx_gemm", "fp8_mx_pack_pow2", "fp8_delayed_quant", "fp8_status_string", "fp8_device_error",
-           "fp8_selftest_bounded_wait")
+           "fp8_mx_gemm", "fp8_mx_pack_pow2", "fp8_delayed_quant", "fp8_block_gemm_quant", "fp8_weight_dequant",
+           "fp8_status_string", "fp8_device_error", "fp8_selftest_bounded_wait")
 
 
 class Fp8Error(RuntimeError):
@@ -60,13 +61,15 @@ def _load() -> ctypes.CDLL:
     L.fp8_mx_gemm.argtypes = [vp, vp, vp, vp, i64, i64, i64, ci, vp, vp]
     L.fp8_mx_pack_pow2.argtypes = [vp, i64, i64, ci, vp, vp]
     L.fp8_delayed_quant.argtypes = [vp, i64, ci, ctypes.c_float, i64, ci, vp, vp, vp, vp, vp, vp, vp]
+    L.fp8_block_gemm_quant.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, ci, ci, vp, vp, vp]
+    L.fp8_weight_dequant.argtypes = [vp, vp, i64, i64, ci, ci, vp, vp]
     L.fp8_status_string.argtypes = [ci]
     L.fp8_status_string.restype = ctypes.c_char_p
     L.fp8_device_error.argtypes = [vp]
     L.fp8_selftest_bounded_wait.argtypes = [i64, vp]
     for name in ("fp8_act_quant", "fp8_weight_quant", "fp8_block_gemm", "fp8_grouped_gemm", "fp8_mx_quant",
-                 "fp8_mx_gemm", "fp8_mx_pack_pow2", "fp8_delayed_quant", "fp8_device_error",
-                 "fp8_selftest_bounded_wait"):
+                 "fp8_mx_gemm", "fp8_mx_pack_pow2", "fp8_delayed_quant", "fp8_block_gemm_quant",
+                 "fp8_weight_dequant", "fp8_device_error", "fp8_selftest_bounded_wait"):
         getattr(L, name).restype = ci
     return L
 
@@ -175,6 +178,42 @@ def fp8_block_gemm(qa: torch.Tensor, sa: torch.Tensor, qw: torch.Tensor, sw: tor
     qa8, qw8, od = _e4m3_codes(qa, "qa"), _e4m3_codes(qw, "qw"), _out_code(y)
     _check("fp8_block_gemm", lib.fp8_block_gemm(_ptr(qa8), _ptr(sa), _ptr(qw8), _ptr(sw), M, N, K,
                                                 od, _ptr(y), _stream(stream)))
+
+
+def fp8_block_gemm_quant(qa: torch.Tensor, sa: torch.Tensor, qw: torch.Tensor, sw: torch.Tensor,
+                         qy: torch.Tensor, sy: torch.Tensor, y: torch.Tensor | None = None, fmt: int = E4M3,
+                         scale_fmt: int = SCALE_FP32, stream=None) -> None:
+    """Block GEMM whose epilogue also quantises its bf16 output for the next layer:
+    qy [M, N] codes and sy [M, N/128] scales equal act_quant(y); y (bf16 [M, N]) is
+    written only when given."""
+    for t in (qa, sa, qw, sw, qy, sy) + ((y,) if y is not None else ()):
+        assert t.is_contiguous()
+    M, K = qa.shape
+    N = qw.shape[0]
+    _expect(qw, (N, K), "qw")
+    _expect(sa, (M, K // 128), "sa", torch.float32)
+    _expect(sw, ((N + 127) // 128, K // 128), "sw", torch.float32)
+    _expect(qy, (M, N), "qy")
+    _expect(sy, (M, N // 128), "sy", torch.float32)
+    if y is not None:
+        _expect(y, (M, N), "y", torch.bfloat16)
+    qa8, qw8 = _e4m3_codes(qa, "qa"), _e4m3_codes(qw, "qw")
+    _check("fp8_block_gemm_quant", lib.fp8_block_gemm_quant(_ptr(qa8), _ptr(sa), _ptr(qw8), _ptr(sw), M, N, K,
+                                                            _ptr(y), fmt, scale_fmt, _ptr(_u8(qy)), _ptr(sy),
+                                                            _stream(stream)))
+
+
+def fp8_weight_dequant(q: torch.Tensor, s_inv: torch.Tensor, w: torch.Tensor, block: int = 128,
+                       fmt: int = E4M3, stream=None) -> None:
+    """FP8 codes q [N, K] with scale_inv (128x128 blocks, or one scale with block=0)
+    -> bf16 w [N, K]."""
+    for t in (q, s_inv, w):
+        assert t.is_contiguous()
+    N, K = q.shape
+    _expect(s_inv, (1,) if block == 0 else ((N + 127) // 128, (K + 127) // 128), "s_inv", torch.float32)
+    _expect(w, (N, K), "w", torch.bfloat16)
+    _check("fp8_weight_dequant", lib.fp8_weight_dequant(_ptr(_u8(q)), _ptr(s_inv), N, K, block, fmt, _ptr(w),
+                                                        _stream(stream)))
 
 
 def fp8_grouped_gemm(qa: torch.Tensor, sa: torch.Tensor, qw: torch.Tensor, sw: torch.Tensor,
@@ -339,3 +378,19 @@ def mx_pack_pow2(s: torch.Tensor, rows: int, K: int, row_block: int, stream=None
     sf = torch.empty((mx_sf_bytes(rows, K),), dtype=torch.uint8, device=s.device)
     fp8_mx_pack_pow2(s, rows, K, row_block, sf, stream)
     return sf
+
+
+def block_gemm_quant(qa, sa, qw, sw, fmt: int = E4M3, scale_fmt: int = SCALE_FP32, with_y: bool = False,
+                     stream=None):
+    M, N = qa.shape[0], qw.shape[0]
+    qy = torch.empty((M, N), dtype=torch.uint8, device=qa.device)
+    sy = torch.empty((M, N // 128), dtype=torch.float32, device=qa.device)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=qa.device) if with_y else None
+    fp8_block_gemm_quant(qa, sa, qw, sw, qy, sy, y, fmt, scale_fmt, stream)
+    return (qy, sy, y) if with_y else (qy, sy)
+
+
+def weight_dequant(q, s_inv, block: int = 128, fmt: int = E4M3, stream=None):
+    w = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
+    fp8_weight_dequant(q, s_inv, w, block, fmt, stream)
+    return w

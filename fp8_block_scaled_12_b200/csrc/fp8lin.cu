@@ -86,14 +86,15 @@ bool launch_regs_ok(K kern) {
   return fa.numRegs == int(kLaunchRegs);
 }
 
-template <int NT, int NBUF, int STAGES, int KB_CAP>
+template <int NT, int NBUF, int STAGES, int KB_CAP, bool QOUT = false>
 int launch_swap(const void* qa, const void* qw, const GemmArgs& a, int64_t w_rows, cudaStream_t st) {
   using C = SwapCfg<NT, NBUF, STAGES, KB_CAP>;
-  constexpr size_t smem = swap_smem_bytes<C>();
+  constexpr size_t smem = swap_smem_bytes<C, QOUT>();
+  static_assert(smem <= 232448, "dynamic shared memory of one CTA (227 KB)");
   CUtensorMap mw, mx;
   if (!make_map_u8(&mw, qw, uint64_t(w_rows), uint64_t(a.K), 128)) return FP8_ERR_CUDA;
   if (!make_map_u8(&mx, qa, uint64_t(a.M > 0 ? a.M : 1), uint64_t(a.K), 32)) return FP8_ERR_CUDA;
-  auto kern = k_gemm_swap<NT, NBUF, STAGES, KB_CAP>;
+  auto kern = k_gemm_swap<NT, NBUF, STAGES, KB_CAP, QOUT>;
   if (!launch_regs_ok(kern)) return FP8_ERR_UNSUPPORTED;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return FP8_ERR_CUDA;
@@ -129,12 +130,13 @@ int launch_mx(const void* qa, const void* qw, const MxArgs& a, cudaStream_t st) 
   return cuda_status(cudaGetLastError());
 }
 
+template <bool QOUT = false>
 int launch_wide(const void* qa, const void* qw, const GemmArgs& a, cudaStream_t st) {
   using C = WideCfg<kWideStages>;
   CUtensorMap ma, mb;
   if (!make_map_u8(&ma, qa, uint64_t(a.M), uint64_t(a.K), C::BM)) return FP8_ERR_CUDA;
   if (!make_map_u8(&mb, qw, uint64_t(a.N), uint64_t(a.K), C::BN)) return FP8_ERR_CUDA;
-  auto kern = k_gemm_wide<kWideStages>;
+  auto kern = k_gemm_wide<kWideStages, QOUT>;
   if (!launch_regs_ok(kern)) return FP8_ERR_UNSUPPORTED;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(C::SMEM));
   if (e != cudaSuccess) return FP8_ERR_CUDA;
@@ -174,6 +176,16 @@ int launch_mx_quant(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, uint8_
   const int64_t warps = (steps + per_warp - 1) / per_warp;
   const int64_t blocks = (warps + 7) / 8;
   k_act_quant<FMT, kScaleUe8m0, U, true><<<int(blocks), 256, 0, st>>>(x, M, K, ldx, q, e8);
+  return cuda_status(cudaGetLastError());
+}
+
+template <int FMT>
+int launch_dequant(const uint8_t* q, const float* s, int64_t N, int64_t K, int block, uint16_t* w, cudaStream_t st) {
+  const int64_t total = N * (K / 16);
+  int64_t blocks = (total + 255) / 256;
+  const int64_t cap = int64_t(num_sms()) * 8;
+  if (blocks > cap) blocks = cap;
+  k_weight_dequant<FMT><<<int(blocks), 256, 0, st>>>(q, s, N, K, block, w);
   return cuda_status(cudaGetLastError());
 }
 
@@ -308,6 +320,42 @@ int fp8_block_gemm(const void* qa, const float* sa, const void* qw, const float*
   if (M <= 64) return launch_swap<64, 4, 8, 56>(qa, qw, a, N, st);
   if (M <= 160) return launch_swap<160, 3, 5, 28>(qa, qw, a, N, st);
   return launch_wide(qa, qw, a, st);
+}
+
+int fp8_block_gemm_quant(const void* qa, const float* sa, const void* qw, const float* sw, int64_t M, int64_t N,
+                         int64_t K, void* y, int fmt, int scale_fmt, void* qy, float* sy, void* stream) {
+  int rc = check_gemm_common(qa, sa, qw, sw, M, N, K, FP8_OUT_BF16, M > 0 ? qy : nullptr);
+  if (rc != FP8_OK) return rc;
+  if (fmt != FP8_E4M3 && fmt != FP8_E5M2) return FP8_ERR_INVALID_ARG;
+  if (scale_fmt != FP8_SCALE_FP32 && scale_fmt != FP8_SCALE_UE8M0) return FP8_ERR_INVALID_ARG;
+  if (N % 128 != 0) return FP8_ERR_SHAPE;                    // whole 128-channel groups
+  if (M == 0) return FP8_OK;
+  if (!qy || !sy) return FP8_ERR_INVALID_ARG;
+  if (!aligned(qy, 16) || !aligned(sy, 4) || (y && !aligned(y, 16))) return FP8_ERR_ALIGNMENT;
+  GemmArgs a{sa, sw, y, nullptr, int(M), int(N), int(K), 1, 0};
+  a.qy = static_cast<uint8_t*>(qy);
+  a.sy = sy;
+  a.qmode = (fmt == FP8_E4M3 ? 0 : 2) + (scale_fmt == FP8_SCALE_UE8M0 ? 1 : 0);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (M <= 64) return launch_swap<64, 4, 8, 56, true>(qa, qw, a, N, st);
+  if (M <= 160) return launch_swap<160, 3, 5, 28, true>(qa, qw, a, N, st);
+  return launch_wide<true>(qa, qw, a, st);
+}
+
+int fp8_weight_dequant(const void* q, const float* s_inv, int64_t N, int64_t K, int block, int fmt, void* w,
+                       void* stream) {
+  if (N < 0 || K <= 0) return FP8_ERR_INVALID_ARG;
+  if (fmt != FP8_E4M3 && fmt != FP8_E5M2) return FP8_ERR_INVALID_ARG;
+  if (block != 128 && block != 0) return FP8_ERR_UNSUPPORTED;
+  if (K % 16 != 0) return FP8_ERR_SHAPE;
+  if (N == 0) return FP8_OK;
+  if (!q || !s_inv || !w) return FP8_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(s_inv, 4) || !aligned(w, 16)) return FP8_ERR_ALIGNMENT;
+  const uint8_t* qb = static_cast<const uint8_t*>(q);
+  uint16_t* wb = static_cast<uint16_t*>(w);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return fmt == FP8_E4M3 ? launch_dequant<kE4M3>(qb, s_inv, N, K, block, wb, st)
+                         : launch_dequant<kE5M2>(qb, s_inv, N, K, block, wb, st);
 }
 
 int fp8_grouped_gemm(const void* qa, const float* sa, const void* qw, const float* sw,

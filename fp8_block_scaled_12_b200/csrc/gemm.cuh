@@ -33,6 +33,7 @@
 #include <cuda_runtime.h>
 
 #include "ptx.cuh"
+#include "quant.cuh"
 
 namespace fp8lin {
 
@@ -52,13 +53,16 @@ static_assert(128 * kProducerRegs + 256 * kConsumerRegs <= 384 * kLaunchRegs, "r
 struct GemmArgs {
   const float* sa;        // [rows][nkb]
   const float* sw;        // [E][nbn][nkb]
-  void* y;                // [rows][N]
+  void* y;                // [rows][N]; may be nullptr when the output is quantised (qy)
   const int32_t* offsets; // grouped: device [E+1]; nullptr = one group [0, M)
   int M;                  // activation rows (total rows for grouped)
   int N;                  // weight rows per expert
   int K;
   int E;
   int out_fp32;
+  uint8_t* qy = nullptr;  // fused act_quant of the bf16 output: codes [M][N]
+  float* sy = nullptr;    //   scales [M][N/128]
+  int qmode = 0;          //   kQE4M3Fp32 / kQE4M3Ue8m0 / kQE5M2Fp32 / kQE5M2Ue8m0
 };
 
 // Shared-memory bookkeeping placed after the stage buffers.
@@ -105,7 +109,9 @@ struct WideCfg {
   static constexpr size_t SMEM = 1024 + size_t(STAGES) * STAGE_BYTES + sizeof(PipeState<STAGES>);
 };
 
-template <int STAGES>
+// QOUT: the epilogue also quantises the bf16 output per (row, 128-column group) for
+// the next layer (args.qy / args.sy / args.qmode); y is then optional.
+template <int STAGES, bool QOUT = false>
 __global__ void __launch_bounds__(kThreads, 1)
     k_gemm_wide(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const GemmArgs args) {
@@ -245,17 +251,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (aborted) break;
       if (row_ok && cols_any) {
+        float amax = 0.0f;
+        if constexpr (QOUT) {
+          // the bf16 output is what the next layer quantises: round in place first
 #pragma unroll
-        for (int j = 0; j < 128; j += 8) {
-          float v[8];
-#pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            const float2 f = unpack2(acc[j / 2 + t]);
-            v[2 * t] = f.x;
-            v[2 * t + 1] = f.y;
+          for (int j = 0; j < 64; ++j) {
+            const float2 f = unpack2(acc[j]);
+            const float lo = __bfloat162float(__float2bfloat16_rn(f.x));
+            const float hi = __bfloat162float(__float2bfloat16_rn(f.y));
+            amax = fmaxf(amax, fmaxf(fabsf(lo), fabsf(hi)));
+            acc[j] = pack2(lo, hi);
           }
-          if (n0 + j < args.N) store8(args.y, out32, m * args.N + n0 + j, v);
         }
+        if (!QOUT || args.y != nullptr) {
+#pragma unroll
+          for (int j = 0; j < 128; j += 8) {
+            float v[8];
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+              const float2 f = unpack2(acc[j / 2 + t]);
+              v[2 * t] = f.x;
+              v[2 * t + 1] = f.y;
+            }
+            if (n0 + j < args.N) store8(args.y, out32, m * args.N + n0 + j, v);
+          }
+        }
+        if constexpr (QOUT)
+          quant_group128_mode(args.qmode, acc, amax, args.qy + m * args.N + n0, args.sy + m * (args.N / 128) + n0 / 128);
       }
     }
   }

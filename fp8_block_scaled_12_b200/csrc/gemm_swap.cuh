@@ -65,13 +65,21 @@ struct alignas(8) SwapState {
   uint64_t tfull[NBUF];
   uint64_t tempty[NBUF];
   uint64_t seg;            // epilogue warps: segment's table loaded, previous one retired
+  uint64_t red[2];         // fused output quantisation: per warpgroup, group maxima exchanged
   uint32_t tmem_base;
   int abort;
 };
 
+// Fused output quantisation: group maxima per warpgroup, [2][4 warps][CW columns].
 template <class C>
+__host__ __device__ constexpr size_t swap_red_bytes() {
+  return size_t(2) * 4 * C::CW * sizeof(float);
+}
+
+template <class C, bool QOUT = false>
 constexpr size_t swap_smem_bytes() {
-  return 1024 + size_t(C::STAGES) * C::STAGE_BYTES + 2 * size_t(C::TBUF_BYTES) + sizeof(SwapState<C::STAGES, C::NBUF>);
+  return 1024 + size_t(C::STAGES) * C::STAGE_BYTES + 2 * size_t(C::TBUF_BYTES) + (QOUT ? swap_red_bytes<C>() : 0) +
+         sizeof(SwapState<C::STAGES, C::NBUF>);
 }
 
 // Rows of expert e: [r0, r1).  offsets == nullptr means one group [0, M).
@@ -139,7 +147,11 @@ __device__ __forceinline__ void swap_seg_load(const GemmArgs& a, const SwapSeg& 
   }
 }
 
-template <int NT, int NBUF, int STAGES, int KB_CAP>
+// QOUT: the epilogue also quantises the bf16 output per (token, 128-row weight block)
+// for the next layer (dense GEMM only; args.qy / args.sy / args.qmode).  A group's 128
+// outputs sit one per thread across a warpgroup, so each warp reduces its 32 and the
+// four warps exchange maxima through shared memory under a bounded mbarrier.
+template <int NT, int NBUF, int STAGES, int KB_CAP, bool QOUT = false>
 __global__ void __launch_bounds__(kThreads, 1)
     k_gemm_swap(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                 const GemmArgs args) {
@@ -150,7 +162,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (base - raw);
   float* table = reinterpret_cast<float*>(gbase + size_t(STAGES) * C::STAGE_BYTES);
-  auto* ps = reinterpret_cast<SwapState<STAGES, NBUF>*>(gbase + size_t(STAGES) * C::STAGE_BYTES + 2 * size_t(C::TBUF_BYTES));
+  float* red = reinterpret_cast<float*>(gbase + size_t(STAGES) * C::STAGE_BYTES + 2 * size_t(C::TBUF_BYTES));
+  auto* ps = reinterpret_cast<SwapState<STAGES, NBUF>*>(gbase + size_t(STAGES) * C::STAGE_BYTES + 2 * size_t(C::TBUF_BYTES) +
+                                                         (QOUT ? swap_red_bytes<C>() : 0));
   volatile int* abort = &ps->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -168,6 +182,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&ps->tempty[b]), kEpiThreads / 32);
     }
     mbar_init(smem_u32(&ps->seg), kEpiThreads / 32);
+    mbar_init(smem_u32(&ps->red[0]), 4);
+    mbar_init(smem_u32(&ps->red[1]), 4);
     ps->abort = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmW);
@@ -251,6 +267,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int col0 = wg * CW;            // first token column of this warpgroup
     const uint32_t table_s = smem_u32(table);
     const uint32_t segbar = smem_u32(&ps->seg);
+    uint32_t rph = 0;                    // phases of this warpgroup's exchange barrier
     SwapSeg cur;
     bool have = swap_seg_find(args, nbn, num_units, blockIdx.x, cur);
     if (have) swap_seg_load<C>(args, cur, nbn, nkb, table_s, ewarp, lane);
@@ -329,7 +346,60 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (aborted) break;
       const int n = (cur.u % nbn) * 128 + quad * 32 + lane;   // weight row of this thread
-      if (cur.seg0 + seglen >= nkb && n < args.N) {
+      if constexpr (QOUT) {
+        if (cur.seg0 + seglen >= nkb) {
+          // the dense fused GEMM has N % 128 == 0, so every thread's row n is valid
+          const int ncols = max(0, min(CW, min(NT, cur.r1 - cur.c0) - col0));
+          float* rw = red + (wg * 4 + quad) * CW;
+#pragma unroll
+          for (int j0 = 0; j0 < CW; j0 += 8) {
+            float mx[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int j = j0 + i;
+              const float2 f = unpack2(acc[j / 2]);
+              const float v = __bfloat162float(__float2bfloat16_rn((j & 1) ? f.y : f.x));
+              acc[j / 2] = (j & 1) ? pack2(f.x, v) : pack2(v, f.y);
+              mx[i] = (j < ncols) ? fabsf(v) : 0.0f;
+            }
+#pragma unroll
+            for (int d = 16; d > 0; d >>= 1)
+#pragma unroll
+              for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], d));
+            if (lane == 0)
+#pragma unroll
+              for (int i = 0; i < 8; ++i) rw[j0 + i] = mx[i];
+          }
+          __syncwarp();
+          const uint32_t rbar = smem_u32(&ps->red[wg]);
+          if (lane == 0) mbar_arrive(rbar);
+          bool rok = mbar_wait(rbar, rph & 1u, abort);
+          ++rph;
+          if (__any_sync(0xffffffffu, !rok)) { aborted = true; break; }
+          const float* rg = red + wg * 4 * CW;
+#pragma unroll
+          for (int j = 0; j < CW; ++j) {       // unrolled: acc stays in registers
+            if (j < ncols) {
+              const float amax = fmaxf(fmaxf(rg[j], rg[CW + j]), fmaxf(rg[2 * CW + j], rg[3 * CW + j]));
+              const float2 f = unpack2(acc[j / 2]);
+              const float v = (j & 1) ? f.y : f.x;
+              float sc;
+              const uint8_t code = quant_one_mode(args.qmode, v, amax, sc);
+              const int64_t tok = cur.c0 + col0 + j;
+              args.qy[tok * args.N + n] = code;
+              if (quad == 0 && lane == 0) args.sy[tok * (args.N / 128) + n / 128] = sc;
+              if (args.y != nullptr)
+                reinterpret_cast<__nv_bfloat16*>(args.y)[tok * args.N + n] = __float2bfloat16_rn(v);
+            }
+          }
+          // the next group's maxima may overwrite the table once all four warps read it
+          __syncwarp();
+          if (lane == 0) mbar_arrive(rbar);
+          rok = mbar_wait(rbar, rph & 1u, abort);
+          ++rph;
+          if (__any_sync(0xffffffffu, !rok)) { aborted = true; break; }
+        }
+      } else if (cur.seg0 + seglen >= nkb && n < args.N) {
         const int ncols = max(0, min(CW, min(NT, cur.r1 - cur.c0) - col0));   // valid token columns
         const int64_t idx0 = int64_t(cur.c0 + col0) * args.N + n;
 #pragma unroll

@@ -21,6 +21,8 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 namespace fp8lin {
@@ -450,6 +452,109 @@ __global__ void k_delayed_finalize(float target, int hist_len, int algo, float* 
     const int np = (p + 1) % hist_len;
     history[np] = 0.0f;
     *pos = np;
+  }
+}
+
+// ------------------------------------------------------ weight dequantisation
+// The BF16 path of the DeepSeek-V3 page (运行时: weight_dequant(weight, weight.scale);
+// FP8 权重转换: fp8_cast_bf16.py): w = bf16(fl32(dec(q) * scale_inv)).  FP8 codes widen
+// exactly to f16 (both E4M3 and E5M2 values are f16 values), then to fp32; one fp32
+// product, one round to nearest even to bf16.  A thread converts 16 codes (one 16-byte
+// load, two 16-byte stores); K % 16 == 0 keeps 16 codes inside one 128-column block.
+template <int FMT>
+__device__ __forceinline__ float2 fp8x2_to_f32(uint16_t two) {
+  uint32_t h2;
+  if (FMT == kE4M3)
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(two));
+  else
+    asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(h2) : "h"(two));
+  const __half2 h = *reinterpret_cast<const __half2*>(&h2);
+  return __half22float2(h);
+}
+
+__device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
+  __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&b);
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(256) k_weight_dequant(const uint8_t* __restrict__ q, const float* __restrict__ s_inv,
+                                                        int64_t N, int64_t K, int block,
+                                                        uint16_t* __restrict__ w) {
+  const int64_t k16 = K / 16, total = N * k16;
+  const int64_t nbk = block > 0 ? (K + block - 1) / block : 1;
+  const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
+    const int64_t n = i / k16, k = (i - n * k16) * 16;
+    const float s = block > 0 ? __ldg(s_inv + (n / block) * nbk + k / block) : __ldg(s_inv);
+    const uint4 c = ldg_stream(reinterpret_cast<const uint4*>(q + n * K + k));
+    const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 a = fp8x2_to_f32<FMT>(uint16_t(cw[j] & 0xFFFFu));
+      const float2 b = fp8x2_to_f32<FMT>(uint16_t(cw[j] >> 16));
+      o[2 * j] = bf16x2_rn(__fmul_rn(a.x, s), __fmul_rn(a.y, s));
+      o[2 * j + 1] = bf16x2_rn(__fmul_rn(b.x, s), __fmul_rn(b.y, s));
+    }
+    uint4* dst = reinterpret_cast<uint4*>(w + n * K + k);
+    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+}
+
+// ------------------------------------------ act_quant of a GEMM output in registers
+// The next layer's activation quantisation fused into a GEMM epilogue: 128 consecutive
+// outputs of one row (one 128-channel group), already rounded to bf16 and held as fp32
+// pairs, are quantised exactly as k_act_quant would quantise that bf16 row: amax,
+// GroupScale, cast.  16-byte code stores; the scale goes to *s.
+template <int FMT, int SF>
+__device__ __forceinline__ void quant_group128(const uint64_t (&v)[64], float amax, uint8_t* q, float* s) {
+  const GroupScale<FMT, SF> sc(amax);
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint32_t lo, hi;
+      asm("mov.b64 {%0, %1}, %2;" : "=r"(lo), "=r"(hi) : "l"(v[c * 8 + 2 * i]));
+      uint32_t lo2, hi2;
+      asm("mov.b64 {%0, %1}, %2;" : "=r"(lo2), "=r"(hi2) : "l"(v[c * 8 + 2 * i + 1]));
+      w[i] = cvt2<FMT>(sc.apply(__uint_as_float(lo)), sc.apply(__uint_as_float(hi))) |
+             (cvt2<FMT>(sc.apply(__uint_as_float(lo2)), sc.apply(__uint_as_float(hi2))) << 16);
+    }
+    *reinterpret_cast<uint4*>(q + 16 * c) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  *s = sc.s;
+}
+
+// Quantisation mode of a fused epilogue: code format and scale format.
+enum : int { kQE4M3Fp32 = 0, kQE4M3Ue8m0 = 1, kQE5M2Fp32 = 2, kQE5M2Ue8m0 = 3 };
+
+__device__ __forceinline__ void quant_group128_mode(int mode, const uint64_t (&v)[64], float amax, uint8_t* q,
+                                                    float* s) {
+  switch (mode) {
+    case kQE4M3Fp32: quant_group128<kE4M3, kScaleFp32>(v, amax, q, s); break;
+    case kQE4M3Ue8m0: quant_group128<kE4M3, kScaleUe8m0>(v, amax, q, s); break;
+    case kQE5M2Fp32: quant_group128<kE5M2, kScaleFp32>(v, amax, q, s); break;
+    default: quant_group128<kE5M2, kScaleUe8m0>(v, amax, q, s); break;
+  }
+}
+
+// One value: scale of its group (computed from the group amax) and its code.
+template <int FMT, int SF>
+__device__ __forceinline__ uint8_t quant_one(float v, float amax, float& s) {
+  const GroupScale<FMT, SF> sc(amax);
+  s = sc.s;
+  return uint8_t(cvt2<FMT>(sc.apply(v), 0.0f) & 0xFFu);
+}
+
+__device__ __forceinline__ uint8_t quant_one_mode(int mode, float v, float amax, float& s) {
+  switch (mode) {
+    case kQE4M3Fp32: return quant_one<kE4M3, kScaleFp32>(v, amax, s);
+    case kQE4M3Ue8m0: return quant_one<kE4M3, kScaleUe8m0>(v, amax, s);
+    case kQE5M2Fp32: return quant_one<kE5M2, kScaleFp32>(v, amax, s);
+    default: return quant_one<kE5M2, kScaleUe8m0>(v, amax, s);
   }
 }
 

@@ -45,7 +45,7 @@ def timed(fn, warm, iters):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--op", required=True, choices=["act_quant", "weight_quant", "gemm", "grouped", "mx_quant",
-                                                    "mx_gemm", "delayed"])
+                                                    "mx_gemm", "delayed", "gemm_quant", "dequant"])
     ap.add_argument("--M", type=int, default=4096)
     ap.add_argument("--N", type=int, default=28672)
     ap.add_argument("--K", type=int, default=8192)
@@ -94,6 +94,24 @@ def main():
         b = qa.numel() + qw.numel() + y.numel() * y.element_size() + sa.numel() * 4 + sw.numel() * 4
         print(f"gemm M={a.M} N={a.N} K={a.K} {a.scale} {a.out}: {ms * 1e3:.2f} us  {fl / ms / 1e9:.1f} TFLOPS  "
               f"{b / ms / 1e6:.1f} GB/s")
+    elif a.op == "gemm_quant":
+        x = synth.activations(a.M, a.K, seed=0, device=dev)
+        w = synth.weights(a.N, a.K, 0.02, seed=0, device=dev)
+        qa, sa = F.act_quant(x, scale_fmt=sf)
+        qw, sw = F.weight_quant(w, scale_fmt=sf)
+        del x, w
+        qy = torch.empty((a.M, a.N), dtype=torch.uint8, device=dev)
+        sy = torch.empty((a.M, a.N // 128), dtype=torch.float32, device=dev)
+        ms = timed(lambda: F.fp8_block_gemm_quant(qa, sa, qw, sw, qy, sy, None, fmt, sf), a.warm, a.iters)
+        fl = 2.0 * a.M * a.N * a.K
+        print(f"gemm_quant M={a.M} N={a.N} K={a.K} {a.scale}: {ms * 1e3:.2f} us  {fl / ms / 1e9:.1f} TFLOPS")
+    elif a.op == "dequant":
+        w = synth.weights(a.M, a.K, 0.02, seed=0, device=dev)
+        q, s = F.weight_quant(w, block=a.block, fmt=fmt, scale_fmt=sf)
+        out = torch.empty_like(w)
+        ms = timed(lambda: F.fp8_weight_dequant(q, s, out, a.block, fmt), a.warm, a.iters)
+        b = a.M * a.K * 3 + s.numel() * 4
+        print(f"dequant N={a.M} K={a.K} block={a.block} {a.fmt}: {ms * 1e3:.2f} us  {b / ms / 1e6:.1f} GB/s")
     elif a.op == "delayed":
         x = synth.activations(a.M, a.K, seed=0, dist=a.dist, device=dev)
         q = torch.empty((a.M, a.K), dtype=torch.uint8, device=dev)

@@ -116,6 +116,37 @@ int fp8_block_gemm(const void* qa, const float* sa, const void* qw, const float*
                    int64_t M, int64_t N, int64_t K, int out_dtype, void* y, void* stream);
 
 /*
+ * fp8_block_gemm_quant -- fp8_block_gemm with bf16 output whose epilogue also applies
+ * the next layer's act_quant to that output (the DeepSeek-V3 page's linear layer runs
+ * act_quant on every linear input, 运行时; here the quantisation of y happens while y is
+ * still in registers instead of in a separate pass over HBM):
+ *   y = fp8_block_gemm(...) rounded to bf16;
+ *   qy, sy = fp8_act_quant(y, group 128, fmt, scale_fmt)   -- bit-exact with it.
+ *
+ *   Arguments as fp8_block_gemm, plus N % 128 == 0 (whole 128-channel groups).
+ *   y      bf16 [M][N], 16-byte aligned, or NULL when only the quantised output is wanted.
+ *   fmt, scale_fmt  as fp8_act_quant.
+ *   qy     codes [M][N], 16-byte aligned; sy fp32 [M][N/128].
+ * Returns FP8_OK or an error status; M == 0 is a no-op.
+ */
+int fp8_block_gemm_quant(const void* qa, const float* sa, const void* qw, const float* sw, int64_t M, int64_t N,
+                         int64_t K, void* y, int fmt, int scale_fmt, void* qy, float* sy, void* stream);
+
+/*
+ * fp8_weight_dequant -- FP8 weights back to bf16, the BF16 path of the DeepSeek-V3 page
+ * (运行时: weight = weight_dequant(weight, weight.scale), then a plain GEMM; FP8 权重转换:
+ * fp8_cast_bf16.py): w[n][k] = bf16_rne(fl32(dec(q[n][k]) * s_inv[n/128][k/128])), or
+ * with the single scale s_inv[0] when block == 0.
+ *
+ *   q      codes [N][K] (fmt), 16-byte aligned; N >= 0, K > 0, K % 16 == 0.
+ *   s_inv  fp32 [ceil(N/128)][ceil(K/128)] (block 128) or [1] (block 0).
+ *   w      bf16 [N][K], 16-byte aligned.
+ * Returns FP8_OK or an error status; N == 0 is a no-op.
+ */
+int fp8_weight_dequant(const void* q, const float* s_inv, int64_t N, int64_t K, int block, int fmt, void* w,
+                       void* stream);
+
+/*
  * fp8_grouped_gemm -- the same GEMM per MoE expert over expert-sorted rows
  * (ROCm page, section 2.3: block-scale fused MoE; DeepSeek-V3 page: 256 routed
  * experts, 8 active per token).  Row m of qa belongs to expert e when

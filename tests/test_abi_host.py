@@ -190,3 +190,21 @@ def test_delayed_quant_validation():
     assert dq(FAKE, 60, 0, F32(400.0), 16, 1, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, S) == SHAPE     # n % 8
     assert dq(FAKE + 8, 64, 0, F32(400.0), 16, 1, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, S) == ALIGN
     assert dq(FAKE, 64, 0, F32(400.0), 16, 1, FAKE, FAKE, FAKE, FAKE, FAKE + 4, FAKE, S) == ALIGN  # uint64 count
+
+
+def test_fused_and_dequant_validation():
+    gq = F.lib.fp8_block_gemm_quant
+    # (qa, sa, qw, sw, M, N, K, y, fmt, scale_fmt, qy, sy, stream)
+    assert gq(FAKE, FAKE, FAKE, FAKE, 16, 272, 256, None, 0, 0, FAKE, FAKE, S) == SHAPE      # N % 128
+    assert gq(FAKE, FAKE, FAKE, FAKE, 16, 256, 200, None, 0, 0, FAKE, FAKE, S) == SHAPE      # K % 128
+    assert gq(FAKE, FAKE, FAKE, FAKE, 16, 256, 256, None, 3, 0, FAKE, FAKE, S) == INVALID    # format
+    assert gq(FAKE, FAKE, FAKE, FAKE, 16, 256, 256, None, 0, 0, FAKE, None, S) == INVALID    # sy
+    assert gq(FAKE, FAKE, FAKE, FAKE, 16, 256, 256, FAKE + 2, 0, 0, FAKE, FAKE, S) == ALIGN  # y
+    assert gq(FAKE, FAKE, FAKE, FAKE, 0, 256, 256, None, 0, 0, None, None, S) == OK
+    dq = F.lib.fp8_weight_dequant
+    # (q, s_inv, N, K, block, fmt, w, stream)
+    assert dq(FAKE, FAKE, 256, 256, 64, 0, FAKE, S) == UNSUP
+    assert dq(FAKE, FAKE, 256, 250, 128, 0, FAKE, S) == SHAPE
+    assert dq(FAKE, FAKE, 256, 256, 128, 4, FAKE, S) == INVALID
+    assert dq(FAKE, FAKE, 256, 256, 128, 0, FAKE + 8, S) == ALIGN
+    assert dq(FAKE, FAKE, 0, 256, 128, 0, None, S) == OK
