@@ -59,6 +59,10 @@ def lib():
         L.orc_mx_quant.argtypes = [vp, i64, i64, i64, i64, ctypes.c_int, vp, vp]
         L.orc_mx_gemm_rows.restype = None
         L.orc_mx_gemm_rows.argtypes = [vp, vp, vp, vp, i64, i64, vp, i64, vp, vp]
+        L.orc_moe_route.restype = None
+        L.orc_moe_route.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp, vp]
+        L.orc_moe_combine_rows.restype = None
+        L.orc_moe_combine_rows.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, i64, vp, vp]
         L.orc_weight_dequant.restype = None
         L.orc_weight_dequant.argtypes = [vp, vp, i64, i64, i64, ctypes.c_int, vp]
         L.orc_delayed_quant.restype = None
@@ -330,3 +334,40 @@ def weight_dequant(q, s_inv, block: int = 128, fmt: int = E4M3, threads: int = 1
 
     _run_parallel(part, _split(N, threads, block if block else 1), threads)
     return out
+
+
+# ------------------------------------------------------------ MoE routing
+def moe_route(scores, k: int):
+    """scores fp32 [T, E] -> dict(ids, w [T, k], offsets [E+1], row_token, row_weight,
+    token_row [T*k])."""
+    sc = np.ascontiguousarray(scores, dtype=np.float32)
+    T, E = sc.shape
+    r = dict(ids=np.empty((T, k), np.int32), w=np.empty((T, k), np.float32), offsets=np.empty(E + 1, np.int32),
+             row_token=np.empty(T * k, np.int32), row_weight=np.empty(T * k, np.float32),
+             token_row=np.empty(T * k, np.int32))
+    lib().orc_moe_route(_ptr(sc), T, E, k, _ptr(r["ids"]), _ptr(r["w"]), _ptr(r["offsets"]), _ptr(r["row_token"]),
+                        _ptr(r["row_weight"]), _ptr(r["token_row"]))
+    return r
+
+
+def moe_combine_rows(qa, sa, qw, sw, ids, w, tokens, threads: int = 1):
+    """fp64 MoE output rows out[t] = sum_j w[t][j] * GEMM(qa[t], expert ids[t][j]) for the
+    listed tokens -> (out [nt, N], bound [nt, N])."""
+    qa = np.ascontiguousarray(qa, dtype=np.uint8)
+    sa = np.ascontiguousarray(sa, dtype=np.float32)
+    qw = np.ascontiguousarray(qw, dtype=np.uint8)
+    sw = np.ascontiguousarray(sw, dtype=np.float32)
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    E, N, K = qw.shape
+    k = ids.shape[1]
+    tokens = np.ascontiguousarray(tokens, dtype=np.int64)
+    out = np.empty((tokens.size, N), np.float64)
+    bound = np.empty((tokens.size, N), np.float64)
+
+    def part(i0, i1):
+        lib().orc_moe_combine_rows(_ptr(qa), _ptr(sa), _ptr(qw), _ptr(sw), _ptr(ids), _ptr(w), k, N, K,
+                                   _ptr(tokens) + i0 * 8, i1 - i0, _ptr(out) + i0 * N * 8, _ptr(bound) + i0 * N * 8)
+
+    _run_parallel(part, _split(tokens.size, threads), threads)
+    return out, bound

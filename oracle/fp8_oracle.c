@@ -42,6 +42,7 @@
 #include <math.h>
 #include <stdint.h>
 #include <stddef.h>
+#include <stdlib.h>
 
 #define ORC_E4M3 0
 #define ORC_E5M2 1
@@ -446,4 +447,84 @@ void orc_weight_dequant(const uint8_t *q, const float *s_inv, int64_t N, int64_t
             out[n * K + k] = orc_round_bf16((double)v);             /* exact widening, one bf16 rounding */
         }
     }
+}
+
+/* ------------------------------------------------------------ MoE routing */
+
+/* Routing and permutation around the grouped GEMM ([P4] 官方配置中最关键的四个参数:
+ * 256 routed experts, n_activated_experts = 8 per token; [P1] 2.3 block-scale fused
+ * MoE).  The pages fix only the counts; the reading taken is the plainest one:
+ *   - each token selects the k experts of largest score (non-negative affinities,
+ *     e.g. sigmoid outputs), in descending score order, a tie going to the lower
+ *     expert index;
+ *   - its gate weights are the selected scores normalised to sum 1: sum = s_0 + ... +
+ *     s_{k-1} accumulated in fp32 in selection order, w_j = fl32(s_j / sum); if the sum
+ *     is 0 every weight is fl32(1 / k);
+ *   - the (token, j) pairs are sorted by (expert, token) -- stable, each token picks an
+ *     expert at most once -- giving offsets [E+1] (rows of expert e are
+ *     [off[e], off[e+1])), row_token / row_weight of every sorted row, and token_row,
+ *     the sorted row of pair (t, j).
+ * ids / w are [T][k]; row_token, row_weight, token_row are [T*k]. */
+void orc_moe_route(const float *scores, int64_t T, int64_t E, int64_t k, int32_t *ids, float *w,
+                   int32_t *offsets, int32_t *row_token, float *row_weight, int32_t *token_row)
+{
+    for (int64_t t = 0; t < T; ++t) {
+        const float *s = scores + t * E;
+        float sum = 0.0f;
+        for (int64_t j = 0; j < k; ++j) {
+            int64_t best = -1;
+            for (int64_t e = 0; e < E; ++e) {
+                int taken = 0;
+                for (int64_t i = 0; i < j; ++i) taken |= (ids[t * k + i] == (int32_t)e);
+                if (taken) continue;
+                if (best < 0 || s[e] > s[best]) best = e;      /* strict: ties keep the lower index */
+            }
+            ids[t * k + j] = (int32_t)best;
+            sum += s[best];
+        }
+        for (int64_t j = 0; j < k; ++j)
+            w[t * k + j] = sum == 0.0f ? 1.0f / (float)k : s[ids[t * k + j]] / sum;
+    }
+    for (int64_t e = 0; e <= E; ++e) offsets[e] = 0;
+    for (int64_t i = 0; i < T * k; ++i) offsets[ids[i] + 1] += 1;
+    for (int64_t e = 0; e < E; ++e) offsets[e + 1] += offsets[e];
+    for (int64_t e = 0; e < E; ++e) {                     /* stable: pairs visited in (t, j) order */
+        int32_t pos = offsets[e];
+        for (int64_t t = 0; t < T; ++t)
+            for (int64_t j = 0; j < k; ++j)
+                if (ids[t * k + j] == (int32_t)e) {
+                    row_token[pos] = (int32_t)t;
+                    row_weight[pos] = w[t * k + j];
+                    token_row[t * k + j] = pos;
+                    ++pos;
+                }
+    }
+}
+
+/* MoE output of selected tokens ([P1] 2.3 fused MoE: expert GEMMs then the gate-weighted
+ * sum): out[t][n] = sum_j w[t][j] * y_j[n], y_j = the block-scaled GEMM of token t's
+ * activation row (qa / sa rows are token-major [T][K]) with expert ids[t][j]'s weights
+ * qw[e] [N][K], sw[e] [N/128][K/128]; fp64, j in order.  bound[t][n] = sum_j |w_j| *
+ * sum_k |a_k w_k| of that expert (the GEMM tolerance scale). */
+void orc_moe_combine_rows(const uint8_t *qa, const float *sa, const uint8_t *qw, const float *sw,
+                          const int32_t *ids, const float *w, int64_t k, int64_t N, int64_t K,
+                          const int64_t *tokens, int64_t nt, double *out, double *bound)
+{
+    const int64_t nkb = K / 128, nbn = (N + 127) / 128;
+    double *y = (double *)malloc(sizeof(double) * (size_t)N);
+    double *b = (double *)malloc(sizeof(double) * (size_t)N);
+    for (int64_t i = 0; i < nt; ++i) {
+        int64_t t = tokens[i];
+        for (int64_t n = 0; n < N; ++n) { out[i * N + n] = 0.0; bound[i * N + n] = 0.0; }
+        for (int64_t j = 0; j < k; ++j) {
+            int64_t e = ids[t * k + j];
+            orc_gemm_rows(qa, sa, qw + e * N * K, sw + e * nbn * nkb, N, K, &t, 1, y, b);
+            for (int64_t n = 0; n < N; ++n) {
+                out[i * N + n] += (double)w[t * k + j] * y[n];
+                bound[i * N + n] += fabs((double)w[t * k + j]) * b[n];
+            }
+        }
+    }
+    free(y);
+    free(b);
 }
