@@ -23,6 +23,7 @@ __all__ = [
     "fp8_act_quant", "fp8_weight_quant", "fp8_block_gemm", "fp8_grouped_gemm", "fp8_mx_quant", "fp8_mx_gemm",
     "fp8_mx_pack_pow2", "fp8_delayed_quant", "DelayedScaling", "AMAX_MOST_RECENT", "AMAX_MAX",
     "fp8_block_gemm_quant", "fp8_weight_dequant", "block_gemm_quant", "weight_dequant",
+    "fp8_moe_route", "fp8_moe_gemm", "moe_route", "moe_gemm",
     "fp8_status_string", "fp8_device_error", "fp8_selftest_bounded_wait",
     "act_quant", "weight_quant", "block_gemm", "grouped_gemm", "mx_quant", "mx_gemm", "mx_pack_pow2",
     "mx_sf_bytes", "EXPORTS",
@@ -39,7 +40,7 @@ FP8_ERR_INVALID_SCALE = 7
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfp8lin.so")
 EXPORTS = ("fp8_act_quant", "fp8_weight_quant", "fp8_block_gemm", "fp8_grouped_gemm", "fp8_mx_quant",
            "fp8_mx_gemm", "fp8_mx_pack_pow2", "fp8_delayed_quant", "fp8_block_gemm_quant", "fp8_weight_dequant",
-           "fp8_status_string", "fp8_device_error", "fp8_selftest_bounded_wait")
+           "fp8_moe_route", "fp8_moe_gemm", "fp8_status_string", "fp8_device_error", "fp8_selftest_bounded_wait")
 
 
 class Fp8Error(RuntimeError):
@@ -63,13 +64,16 @@ def _load() -> ctypes.CDLL:
     L.fp8_delayed_quant.argtypes = [vp, i64, ci, ctypes.c_float, i64, ci, vp, vp, vp, vp, vp, vp, vp]
     L.fp8_block_gemm_quant.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, ci, ci, vp, vp, vp]
     L.fp8_weight_dequant.argtypes = [vp, vp, i64, i64, ci, ci, vp, vp]
+    L.fp8_moe_route.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp, vp, vp]
+    L.fp8_moe_gemm.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, vp, vp]
     L.fp8_status_string.argtypes = [ci]
     L.fp8_status_string.restype = ctypes.c_char_p
     L.fp8_device_error.argtypes = [vp]
     L.fp8_selftest_bounded_wait.argtypes = [i64, vp]
     for name in ("fp8_act_quant", "fp8_weight_quant", "fp8_block_gemm", "fp8_grouped_gemm", "fp8_mx_quant",
                  "fp8_mx_gemm", "fp8_mx_pack_pow2", "fp8_delayed_quant", "fp8_block_gemm_quant",
-                 "fp8_weight_dequant", "fp8_device_error", "fp8_selftest_bounded_wait"):
+                 "fp8_weight_dequant", "fp8_moe_route", "fp8_moe_gemm", "fp8_device_error",
+                 "fp8_selftest_bounded_wait"):
         getattr(L, name).restype = ci
     return L
 
@@ -214,6 +218,45 @@ def fp8_weight_dequant(q: torch.Tensor, s_inv: torch.Tensor, w: torch.Tensor, bl
     _expect(w, (N, K), "w", torch.bfloat16)
     _check("fp8_weight_dequant", lib.fp8_weight_dequant(_ptr(_u8(q)), _ptr(s_inv), N, K, block, fmt, _ptr(w),
                                                         _stream(stream)))
+
+
+def fp8_moe_route(scores: torch.Tensor, k: int, ids: torch.Tensor, w: torch.Tensor, offsets: torch.Tensor,
+                  row_token: torch.Tensor, row_weight: torch.Tensor, token_row: torch.Tensor, stream=None) -> None:
+    """Top-k routing of fp32 scores [T, E], gate weights, and the stable expert sort."""
+    for t in (scores, ids, w, offsets, row_token, row_weight, token_row):
+        assert t.is_contiguous()
+    T, E = scores.shape
+    _expect(scores, (T, E), "scores", torch.float32)
+    _expect(ids, (T, k), "ids", torch.int32)
+    _expect(w, (T, k), "w", torch.float32)
+    _expect(offsets, (E + 1,), "offsets", torch.int32)
+    for t, n, d in ((row_token, "row_token", torch.int32), (row_weight, "row_weight", torch.float32),
+                    (token_row, "token_row", torch.int32)):
+        _expect(t, (T * k,), n, d)
+    _check("fp8_moe_route", lib.fp8_moe_route(_ptr(scores), T, E, k, _ptr(ids), _ptr(w), _ptr(offsets),
+                                              _ptr(row_token), _ptr(row_weight), _ptr(token_row), _stream(stream)))
+
+
+def fp8_moe_gemm(qa: torch.Tensor, sa: torch.Tensor, qw: torch.Tensor, sw: torch.Tensor, route: dict,
+                 out: torch.Tensor, stream=None) -> None:
+    """MoE expert GEMMs over routed rows: token-major qa [T, K] / sa [T, K/128] are
+    gathered per expert, and out fp32 [T, N] = sum_j w[t, j] * expert_j(qa[t])."""
+    for t in (qa, sa, qw, sw, out):
+        assert t.is_contiguous()
+    T, K = qa.shape
+    E, N, _ = qw.shape
+    k = route["ids"].shape[1]
+    _expect(qw, (E, N, K), "qw")
+    _expect(sa, (T, K // 128), "sa", torch.float32)
+    _expect(sw, (E, (N + 127) // 128, K // 128), "sw", torch.float32)
+    _expect(route["offsets"], (E + 1,), "offsets", torch.int32)
+    _expect(route["row_token"], (T * k,), "row_token", torch.int32)
+    _expect(route["row_weight"], (T * k,), "row_weight", torch.float32)
+    _expect(out, (T, N), "out", torch.float32)
+    qa8, qw8 = _e4m3_codes(qa, "qa"), _e4m3_codes(qw, "qw")
+    _check("fp8_moe_gemm", lib.fp8_moe_gemm(_ptr(qa8), _ptr(sa), _ptr(qw8), _ptr(sw), _ptr(route["offsets"]),
+                                            _ptr(route["row_token"]), _ptr(route["row_weight"]), T, E, k, N, K,
+                                            _ptr(out), _stream(stream)))
 
 
 def fp8_grouped_gemm(qa: torch.Tensor, sa: torch.Tensor, qw: torch.Tensor, sw: torch.Tensor,
@@ -394,3 +437,22 @@ def weight_dequant(q, s_inv, block: int = 128, fmt: int = E4M3, stream=None):
     w = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
     fp8_weight_dequant(q, s_inv, w, block, fmt, stream)
     return w
+
+
+def moe_route(scores: torch.Tensor, k: int, stream=None) -> dict:
+    T, E = scores.shape
+    dev = scores.device
+    r = dict(ids=torch.empty((T, k), dtype=torch.int32, device=dev),
+             w=torch.empty((T, k), dtype=torch.float32, device=dev),
+             offsets=torch.empty((E + 1,), dtype=torch.int32, device=dev),
+             row_token=torch.empty((T * k,), dtype=torch.int32, device=dev),
+             row_weight=torch.empty((T * k,), dtype=torch.float32, device=dev),
+             token_row=torch.empty((T * k,), dtype=torch.int32, device=dev))
+    fp8_moe_route(scores, k, r["ids"], r["w"], r["offsets"], r["row_token"], r["row_weight"], r["token_row"], stream)
+    return r
+
+
+def moe_gemm(qa, sa, qw, sw, route: dict, stream=None):
+    out = torch.empty((qa.shape[0], qw.shape[1]), dtype=torch.float32, device=qa.device)
+    fp8_moe_gemm(qa, sa, qw, sw, route, out, stream)
+    return out

@@ -17,7 +17,7 @@ CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libfp8lin.so")
 SOURCES = ["fp8lin.cu"]
-DEPS = ["fp8lin.cu", "gemm.cuh", "gemm_mx.cuh", "gemm_swap.cuh", "quant.cuh", "ptx.cuh"]
+DEPS = ["fp8lin.cu", "gemm.cuh", "gemm_mx.cuh", "gemm_swap.cuh", "moe.cuh", "quant.cuh", "ptx.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 

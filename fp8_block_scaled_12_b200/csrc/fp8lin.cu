@@ -11,6 +11,7 @@
 #include "gemm.cuh"
 #include "gemm_mx.cuh"
 #include "gemm_swap.cuh"
+#include "moe.cuh"
 #include "ptx.cuh"
 #include "quant.cuh"
 
@@ -86,15 +87,17 @@ bool launch_regs_ok(K kern) {
   return fa.numRegs == int(kLaunchRegs);
 }
 
-template <int NT, int NBUF, int STAGES, int KB_CAP, bool QOUT = false>
+template <int NT, int NBUF, int STAGES, int KB_CAP, bool QOUT = false, bool MOE = false>
 int launch_swap(const void* qa, const void* qw, const GemmArgs& a, int64_t w_rows, cudaStream_t st) {
   using C = SwapCfg<NT, NBUF, STAGES, KB_CAP>;
   constexpr size_t smem = swap_smem_bytes<C, QOUT>();
   static_assert(smem <= 232448, "dynamic shared memory of one CTA (227 KB)");
   CUtensorMap mw, mx;
   if (!make_map_u8(&mw, qw, uint64_t(w_rows), uint64_t(a.K), 128)) return FP8_ERR_CUDA;
-  if (!make_map_u8(&mx, qa, uint64_t(a.M > 0 ? a.M : 1), uint64_t(a.K), 32)) return FP8_ERR_CUDA;
-  auto kern = k_gemm_swap<NT, NBUF, STAGES, KB_CAP, QOUT>;
+  // MOE: token-major qa of T rows read by one-row gathers; otherwise the rows in order
+  const uint64_t xrows = uint64_t(MOE ? a.moe_T : (a.M > 0 ? a.M : 1));
+  if (!make_map_u8(&mx, qa, xrows, uint64_t(a.K), MOE ? 1u : 32u)) return FP8_ERR_CUDA;
+  auto kern = k_gemm_swap<NT, NBUF, STAGES, KB_CAP, QOUT, MOE>;
   if (!launch_regs_ok(kern)) return FP8_ERR_UNSUPPORTED;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return FP8_ERR_CUDA;
@@ -446,6 +449,53 @@ int fp8_mx_pack_pow2(const float* s, int64_t rows, int64_t K, int row_block, voi
   k_mx_pack_pow2<<<unsigned((n + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
       s, rows, nkb, row_block, static_cast<uint8_t*>(sf));
   return cuda_status(cudaGetLastError());
+}
+
+int fp8_moe_route(const float* scores, int64_t T, int64_t E, int64_t k, int32_t* ids, float* w, int32_t* offsets,
+                  int32_t* row_token, float* row_weight, int32_t* token_row, void* stream) {
+  if (T < 0 || E < 1 || E > kMoeMaxE || k < 1 || k > kMoeMaxK || k > E) return FP8_ERR_INVALID_ARG;
+  if (T * k > INT32_MAX) return FP8_ERR_SHAPE;
+  if (!offsets) return FP8_ERR_INVALID_ARG;
+  if (T > 0 && (!scores || !ids || !w || !row_token || !row_weight || !token_row)) return FP8_ERR_INVALID_ARG;
+  if (!aligned(scores, 4) || !aligned(ids, 4) || !aligned(w, 4) || !aligned(offsets, 4) || !aligned(row_token, 4) ||
+      !aligned(row_weight, 4) || !aligned(token_row, 4))
+    return FP8_ERR_ALIGNMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (T > 0) {
+    const int blocks = int((T * 32 + 255) / 256);
+    if (E <= 256)
+      k_moe_topk<8><<<blocks, 256, 0, st>>>(scores, int(T), int(E), int(k), ids, w);
+    else
+      k_moe_topk<32><<<blocks, 256, 0, st>>>(scores, int(T), int(E), int(k), ids, w);
+    if (cudaGetLastError() != cudaSuccess) return FP8_ERR_CUDA;
+  }
+  const size_t smem = size_t(32) * size_t(E) * sizeof(int32_t);
+  if (cudaFuncSetAttribute(k_moe_sort, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
+    return FP8_ERR_CUDA;
+  k_moe_sort<<<1, 1024, smem, st>>>(ids, w, int(T), int(E), int(k), offsets, row_token, row_weight, token_row);
+  return cuda_status(cudaGetLastError());
+}
+
+int fp8_moe_gemm(const void* qa, const float* sa, const void* qw, const float* sw, const int32_t* offsets,
+                 const int32_t* row_token, const float* row_weight, int64_t T, int64_t E, int64_t k, int64_t N,
+                 int64_t K, float* out, void* stream) {
+  if (T < 0 || E <= 0 || k <= 0 || N <= 0 || K <= 0) return FP8_ERR_INVALID_ARG;
+  if (K % 128 != 0 || N % 16 != 0) return FP8_ERR_SHAPE;
+  if (T * k > INT32_MAX || E * N > INT32_MAX || K > INT32_MAX || T * N > (int64_t(1) << 40)) return FP8_ERR_SHAPE;
+  if (!qw || !sw || !offsets || !out) return FP8_ERR_INVALID_ARG;
+  if (T > 0 && (!qa || !sa || !row_token || !row_weight)) return FP8_ERR_INVALID_ARG;
+  if (!aligned(qw, 16) || !aligned(sw, 4) || !aligned(offsets, 4) || !aligned(out, 4)) return FP8_ERR_ALIGNMENT;
+  if (T > 0 && (!aligned(qa, 16) || !aligned(sa, 4) || !aligned(row_token, 4) || !aligned(row_weight, 4)))
+    return FP8_ERR_ALIGNMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (T == 0) return FP8_OK;
+  if (cudaMemsetAsync(out, 0, size_t(T) * size_t(N) * sizeof(float), st) != cudaSuccess) return FP8_ERR_CUDA;
+  GemmArgs a{sa, sw, nullptr, offsets, int(T * k), int(N), int(K), int(E), 1};
+  a.row_token = row_token;
+  a.row_weight = row_weight;
+  a.moe_out = out;
+  a.moe_T = int(T);
+  return launch_swap<160, 3, 5, 28, false, true>(qa, qw, a, E * N, st);
 }
 
 int fp8_selftest_bounded_wait(int64_t limit_ns, void* stream) {

@@ -45,7 +45,7 @@ def timed(fn, warm, iters):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--op", required=True, choices=["act_quant", "weight_quant", "gemm", "grouped", "mx_quant",
-                                                    "mx_gemm", "delayed", "gemm_quant", "dequant"])
+                                                    "mx_gemm", "delayed", "gemm_quant", "dequant", "moe"])
     ap.add_argument("--M", type=int, default=4096)
     ap.add_argument("--N", type=int, default=28672)
     ap.add_argument("--K", type=int, default=8192)
@@ -94,6 +94,22 @@ def main():
         b = qa.numel() + qw.numel() + y.numel() * y.element_size() + sa.numel() * 4 + sw.numel() * 4
         print(f"gemm M={a.M} N={a.N} K={a.K} {a.scale} {a.out}: {ms * 1e3:.2f} us  {fl / ms / 1e9:.1f} TFLOPS  "
               f"{b / ms / 1e6:.1f} GB/s")
+    elif a.op == "moe":
+        # routed layer: scores -> route, act_quant of the tokens, gather GEMM + weighted scatter
+        g = torch.Generator(device=dev).manual_seed(3)
+        scores = torch.rand((a.tokens, a.E), generator=g, device=dev, dtype=torch.float32)
+        x = synth.activations(a.tokens, a.K, seed=0, device=dev)
+        qa, sa = F.act_quant(x)
+        qw = torch.empty((a.E, a.N, a.K), dtype=torch.uint8, device=dev)
+        sw = torch.empty((a.E, (a.N + 127) // 128, a.K // 128), dtype=torch.float32, device=dev)
+        for e in range(a.E):
+            F.fp8_weight_quant(synth.weights(a.N, a.K, 0.02, seed=0, chunk=e, device=dev), qw[e], sw[e])
+        route = F.moe_route(scores, a.topk)
+        out = torch.empty((a.tokens, a.N), dtype=torch.float32, device=dev)
+        ms = timed(lambda: F.fp8_moe_gemm(qa, sa, qw, sw, route, out), a.warm, a.iters)
+        fl = 2.0 * a.tokens * a.topk * a.N * a.K
+        print(f"moe_gemm tokens={a.tokens} E={a.E} top-{a.topk} N={a.N} K={a.K}: {ms * 1e3:.1f} us  "
+              f"{fl / ms / 1e9:.1f} TFLOPS")
     elif a.op == "gemm_quant":
         x = synth.activations(a.M, a.K, seed=0, device=dev)
         w = synth.weights(a.N, a.K, 0.02, seed=0, device=dev)

@@ -208,3 +208,21 @@ def test_fused_and_dequant_validation():
     assert dq(FAKE, FAKE, 256, 256, 128, 4, FAKE, S) == INVALID
     assert dq(FAKE, FAKE, 256, 256, 128, 0, FAKE + 8, S) == ALIGN
     assert dq(FAKE, FAKE, 0, 256, 128, 0, None, S) == OK
+
+
+def test_moe_validation():
+    mr = F.lib.fp8_moe_route
+    # (scores, T, E, k, ids, w, offsets, row_token, row_weight, token_row, stream)
+    assert mr(FAKE, 16, 0, 2, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, S) == INVALID       # E
+    assert mr(FAKE, 16, 2048, 8, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, S) == INVALID    # E > 1024
+    assert mr(FAKE, 16, 8, 9, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, S) == INVALID       # k > E
+    assert mr(FAKE, 16, 8, 33, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, S) == INVALID      # k > 32
+    assert mr(FAKE + 2, 16, 8, 2, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, S) == ALIGN
+    mg = F.lib.fp8_moe_gemm
+    # (qa, sa, qw, sw, offsets, row_token, row_weight, T, E, k, N, K, out, stream)
+    assert mg(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 16, 4, 2, 256, 200, FAKE, S) == SHAPE   # K % 128
+    assert mg(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 16, 4, 2, 250, 256, FAKE, S) == SHAPE   # N % 16
+    assert mg(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 16, 0, 2, 256, 256, FAKE, S) == INVALID
+    assert mg(FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, 16, 4, 2, 256, 256, FAKE, S) == INVALID
+    assert mg(FAKE + 8, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 16, 4, 2, 256, 256, FAKE, S) == ALIGN
+    assert mg(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 4, 2, 256, 256, FAKE, S) == OK
