@@ -413,21 +413,21 @@ def measure_rows(dev, peaks):
     # expert GEMMs gathering their rows and adding gate-weighted outputs per token
     g = torch.Generator(device=dev).manual_seed(3)
     scores = torch.rand((p["T"], E), generator=g, device=dev, dtype=torch.float32)
-    qt, st_ = F.act_quant(xt)
     route = F.moe_route(scores, p["topk"])
+    qt, st_ = F.act_quant_permute(xt, route)
     out = torch.empty((p["T"], N), dtype=torch.float32, device=dev)
 
     def moe_step():
         F.fp8_moe_route(scores, p["topk"], route["ids"], route["w"], route["offsets"], route["row_token"],
                         route["row_weight"], route["token_row"])
-        F.fp8_act_quant(xt, qt, st_)
+        F.fp8_act_quant_permute(xt, route, qt, st_)
         F.fp8_moe_gemm(qt, st_, qwe, swe, route, out)
 
     ms_f = time_launches(moe_step, 5)
     ms_r = time_launches(lambda: F.fp8_moe_route(scores, p["topk"], route["ids"], route["w"], route["offsets"],
                                                  route["row_token"], route["row_weight"], route["token_row"]), 10)
     fl_m = 2.0 * p["T"] * p["topk"] * N * K
-    res["moe layer fused (route + act_quant + gather GEMM + weighted scatter) 4096 tok top-8/256"] = {
+    res["moe layer (route + act_quant_permute + GEMM with weighted scatter) 4096 tok top-8/256"] = {
         "us": round(ms_f * 1e3, 1), "TFLOPS": round(fl_m / ms_f / 1e9, 1), "route_us": round(ms_r * 1e3, 1)}
     del out, route, scores
     ms = time_launches(lambda: F.fp8_grouped_gemm(qa, sa, qwe, swe, offd, y), 5)

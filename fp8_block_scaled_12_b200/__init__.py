@@ -23,7 +23,7 @@ __all__ = [
     "fp8_act_quant", "fp8_weight_quant", "fp8_block_gemm", "fp8_grouped_gemm", "fp8_mx_quant", "fp8_mx_gemm",
     "fp8_mx_pack_pow2", "fp8_delayed_quant", "DelayedScaling", "AMAX_MOST_RECENT", "AMAX_MAX",
     "fp8_block_gemm_quant", "fp8_weight_dequant", "block_gemm_quant", "weight_dequant",
-    "fp8_moe_route", "fp8_moe_gemm", "moe_route", "moe_gemm",
+    "fp8_moe_route", "fp8_moe_gemm", "fp8_act_quant_permute", "moe_route", "moe_gemm", "act_quant_permute",
     "fp8_status_string", "fp8_device_error", "fp8_selftest_bounded_wait",
     "act_quant", "weight_quant", "block_gemm", "grouped_gemm", "mx_quant", "mx_gemm", "mx_pack_pow2",
     "mx_sf_bytes", "EXPORTS",
@@ -40,7 +40,8 @@ FP8_ERR_INVALID_SCALE = 7
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfp8lin.so")
 EXPORTS = ("fp8_act_quant", "fp8_weight_quant", "fp8_block_gemm", "fp8_grouped_gemm", "fp8_mx_quant",
            "fp8_mx_gemm", "fp8_mx_pack_pow2", "fp8_delayed_quant", "fp8_block_gemm_quant", "fp8_weight_dequant",
-           "fp8_moe_route", "fp8_moe_gemm", "fp8_status_string", "fp8_device_error", "fp8_selftest_bounded_wait")
+           "fp8_moe_route", "fp8_moe_gemm", "fp8_act_quant_permute", "fp8_status_string", "fp8_device_error",
+           "fp8_selftest_bounded_wait")
 
 
 class Fp8Error(RuntimeError):
@@ -66,14 +67,15 @@ def _load() -> ctypes.CDLL:
     L.fp8_weight_dequant.argtypes = [vp, vp, i64, i64, ci, ci, vp, vp]
     L.fp8_moe_route.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp, vp, vp]
     L.fp8_moe_gemm.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, vp, vp]
+    L.fp8_act_quant_permute.argtypes = [vp, i64, i64, i64, ci, ci, vp, i64, vp, vp, vp]
     L.fp8_status_string.argtypes = [ci]
     L.fp8_status_string.restype = ctypes.c_char_p
     L.fp8_device_error.argtypes = [vp]
     L.fp8_selftest_bounded_wait.argtypes = [i64, vp]
     for name in ("fp8_act_quant", "fp8_weight_quant", "fp8_block_gemm", "fp8_grouped_gemm", "fp8_mx_quant",
                  "fp8_mx_gemm", "fp8_mx_pack_pow2", "fp8_delayed_quant", "fp8_block_gemm_quant",
-                 "fp8_weight_dequant", "fp8_moe_route", "fp8_moe_gemm", "fp8_device_error",
-                 "fp8_selftest_bounded_wait"):
+                 "fp8_weight_dequant", "fp8_moe_route", "fp8_moe_gemm", "fp8_act_quant_permute",
+                 "fp8_device_error", "fp8_selftest_bounded_wait"):
         getattr(L, name).restype = ci
     return L
 
@@ -237,17 +239,33 @@ def fp8_moe_route(scores: torch.Tensor, k: int, ids: torch.Tensor, w: torch.Tens
                                               _ptr(row_token), _ptr(row_weight), _ptr(token_row), _stream(stream)))
 
 
+def fp8_act_quant_permute(x: torch.Tensor, route: dict, q: torch.Tensor, s: torch.Tensor, fmt: int = E4M3,
+                          scale_fmt: int = SCALE_FP32, stream=None) -> None:
+    """act_quant of bf16 x [T, K] with each token's codes / scales written to its k
+    expert-sorted rows (q [T*k, K], s [T*k, ceil(K/128)])."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    T, K = x.shape
+    k = route["ids"].shape[1]
+    _expect(route["token_row"], (T * k,), "token_row", torch.int32)
+    _expect(q, (T * k, K), "q")
+    _expect(s, (T * k, (K + 127) // 128), "s", torch.float32)
+    _check("fp8_act_quant_permute", lib.fp8_act_quant_permute(_ptr(x), T, K, x.stride(0), fmt, scale_fmt,
+                                                              _ptr(route["token_row"]), k, _ptr(_u8(q)), _ptr(s),
+                                                              _stream(stream)))
+
+
 def fp8_moe_gemm(qa: torch.Tensor, sa: torch.Tensor, qw: torch.Tensor, sw: torch.Tensor, route: dict,
                  out: torch.Tensor, stream=None) -> None:
-    """MoE expert GEMMs over routed rows: token-major qa [T, K] / sa [T, K/128] are
-    gathered per expert, and out fp32 [T, N] = sum_j w[t, j] * expert_j(qa[t])."""
+    """Expert GEMMs over the expert-sorted rows qa [T*k, K] / sa [T*k, K/128]
+    (act_quant_permute) with the gate-weighted combine fused: out fp32 [T, N]."""
     for t in (qa, sa, qw, sw, out):
         assert t.is_contiguous()
-    T, K = qa.shape
+    R, K = qa.shape
     E, N, _ = qw.shape
-    k = route["ids"].shape[1]
+    T, k = route["ids"].shape
+    _expect(qa, (T * k, K), "qa")
     _expect(qw, (E, N, K), "qw")
-    _expect(sa, (T, K // 128), "sa", torch.float32)
+    _expect(sa, (T * k, K // 128), "sa", torch.float32)
     _expect(sw, (E, (N + 127) // 128, K // 128), "sw", torch.float32)
     _expect(route["offsets"], (E + 1,), "offsets", torch.int32)
     _expect(route["row_token"], (T * k,), "row_token", torch.int32)
@@ -452,7 +470,16 @@ def moe_route(scores: torch.Tensor, k: int, stream=None) -> dict:
     return r
 
 
+def act_quant_permute(x: torch.Tensor, route: dict, fmt: int = E4M3, scale_fmt: int = SCALE_FP32, stream=None):
+    T, K = x.shape
+    k = route["ids"].shape[1]
+    q = torch.empty((T * k, K), dtype=torch.uint8, device=x.device)
+    s = torch.empty((T * k, (K + 127) // 128), dtype=torch.float32, device=x.device)
+    fp8_act_quant_permute(x, route, q, s, fmt, scale_fmt, stream)
+    return q, s
+
+
 def moe_gemm(qa, sa, qw, sw, route: dict, stream=None):
-    out = torch.empty((qa.shape[0], qw.shape[1]), dtype=torch.float32, device=qa.device)
+    out = torch.empty((route["ids"].shape[0], qw.shape[1]), dtype=torch.float32, device=qa.device)
     fp8_moe_gemm(qa, sa, qw, sw, route, out, stream)
     return out

@@ -94,9 +94,7 @@ int launch_swap(const void* qa, const void* qw, const GemmArgs& a, int64_t w_row
   static_assert(smem <= 232448, "dynamic shared memory of one CTA (227 KB)");
   CUtensorMap mw, mx;
   if (!make_map_u8(&mw, qw, uint64_t(w_rows), uint64_t(a.K), 128)) return FP8_ERR_CUDA;
-  // MOE: token-major qa of T rows read by one-row gathers; otherwise the rows in order
-  const uint64_t xrows = uint64_t(MOE ? a.moe_T : (a.M > 0 ? a.M : 1));
-  if (!make_map_u8(&mx, qa, xrows, uint64_t(a.K), MOE ? 1u : 32u)) return FP8_ERR_CUDA;
+  if (!make_map_u8(&mx, qa, uint64_t(a.M > 0 ? a.M : 1), uint64_t(a.K), 32)) return FP8_ERR_CUDA;
   auto kern = k_gemm_swap<NT, NBUF, STAGES, KB_CAP, QOUT, MOE>;
   if (!launch_regs_ok(kern)) return FP8_ERR_UNSUPPORTED;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
@@ -165,6 +163,20 @@ int launch_act_quant(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, uint8
   const int64_t warps = (steps + per_warp - 1) / per_warp;
   const int64_t blocks = (warps + 7) / 8;
   k_act_quant<FMT, SF, U><<<int(blocks), 256, 0, st>>>(x, M, K, ldx, q, s);
+  return cuda_status(cudaGetLastError());
+}
+
+template <int FMT, int SF>
+int launch_act_quant_permute(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q, float* s,
+                             const int32_t* perm, int k, cudaStream_t st) {
+  constexpr int U = 2;
+  const int64_t items = M * ((K + 127) / 128);
+  const int64_t steps = (items + 8 * U - 1) / (8 * U);
+  const int64_t max_warps = int64_t(num_sms()) * 8 * (256 / 32);
+  const int64_t per_warp = (steps + max_warps - 1) / max_warps;
+  const int64_t warps = (steps + per_warp - 1) / per_warp;
+  const int64_t blocks = (warps + 7) / 8;
+  k_act_quant<FMT, SF, U, false, true><<<int(blocks), 256, 0, st>>>(x, M, K, ldx, q, s, perm, k, M * k);
   return cuda_status(cudaGetLastError());
 }
 
@@ -474,6 +486,28 @@ int fp8_moe_route(const float* scores, int64_t T, int64_t E, int64_t k, int32_t*
     return FP8_ERR_CUDA;
   k_moe_sort<<<1, 1024, smem, st>>>(ids, w, int(T), int(E), int(k), offsets, row_token, row_weight, token_row);
   return cuda_status(cudaGetLastError());
+}
+
+int fp8_act_quant_permute(const void* x, int64_t T, int64_t K, int64_t ldx, int fmt, int scale_fmt,
+                          const int32_t* token_row, int64_t k, void* q, float* s, void* stream) {
+  if (T < 0 || K <= 0 || ldx < K || k < 1 || k > kMoeMaxK) return FP8_ERR_INVALID_ARG;
+  if (fmt != FP8_E4M3 && fmt != FP8_E5M2) return FP8_ERR_INVALID_ARG;
+  if (scale_fmt != FP8_SCALE_FP32 && scale_fmt != FP8_SCALE_UE8M0) return FP8_ERR_INVALID_ARG;
+  if (K % 16 != 0) return FP8_ERR_SHAPE;
+  if (T * k > INT32_MAX) return FP8_ERR_SHAPE;
+  if (T == 0) return FP8_OK;
+  if (!x || !q || !s || !token_row) return FP8_ERR_INVALID_ARG;
+  if (ldx % 8 != 0 || !aligned(x, 16) || !aligned(q, 16) || !aligned(s, 4) || !aligned(token_row, 4))
+    return FP8_ERR_ALIGNMENT;
+  const uint16_t* xb = static_cast<const uint16_t*>(x);
+  uint8_t* qb = static_cast<uint8_t*>(q);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int kk = int(k);
+  if (fmt == FP8_E4M3)
+    return scale_fmt == FP8_SCALE_FP32 ? launch_act_quant_permute<kE4M3, kScaleFp32>(xb, T, K, ldx, qb, s, token_row, kk, st)
+                                       : launch_act_quant_permute<kE4M3, kScaleUe8m0>(xb, T, K, ldx, qb, s, token_row, kk, st);
+  return scale_fmt == FP8_SCALE_FP32 ? launch_act_quant_permute<kE5M2, kScaleFp32>(xb, T, K, ldx, qb, s, token_row, kk, st)
+                                     : launch_act_quant_permute<kE5M2, kScaleUe8m0>(xb, T, K, ldx, qb, s, token_row, kk, st);
 }
 
 int fp8_moe_gemm(const void* qa, const float* sa, const void* qw, const float* sw, const int32_t* offsets,

@@ -63,9 +63,8 @@ struct GemmArgs {
   uint8_t* qy = nullptr;  // fused act_quant of the bf16 output: codes [M][N]
   float* sy = nullptr;    //   scales [M][N/128]
   int qmode = 0;          //   kQE4M3Fp32 / kQE4M3Ue8m0 / kQE5M2Fp32 / kQE5M2Ue8m0
-  // MoE gather / scatter (grouped GEMM over routed rows): row r of the expert-sorted
-  // order reads token row_token[r] of the token-major qa / sa (T rows) and its output
-  // is added, times row_weight[r], into moe_out[token] (fp32 [T][N]).
+  // MoE scatter (grouped GEMM over expert-sorted rows): the output of sorted row r is
+  // added, times row_weight[r], into moe_out[row_token[r]] (fp32 [T][N]).
   const int32_t* row_token = nullptr;
   const float* row_weight = nullptr;
   float* moe_out = nullptr;

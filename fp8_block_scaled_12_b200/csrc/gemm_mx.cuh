@@ -47,7 +47,7 @@ enum : int { kSfE8m0x32 = 0, kSfPow2x128 = 1 };
 
 // Register split of this kernel: its epilogue holds one tile's accumulator slice (at
 // most 128 values) rather than 128 running sums plus staged partials, so the
-// producer warpgroup (TMA, MMA issue, scale gathering) gets more registers than in
+// producer warpgroup (TMA and MMA issue) gets more registers than in
 // the promotion kernels.  128 * 104 + 256 * 200 == 384 * kLaunchRegs.
 constexpr uint32_t kMxProducerRegs = 104;
 constexpr uint32_t kMxConsumerRegs = 200;

@@ -132,23 +132,21 @@ __device__ __forceinline__ bool swap_seg_next(const GemmArgs& a, int nbn, int nu
 
 // All 256 epilogue threads: start the copies of segment s's scales into the table at
 // shared address `tbl`: row kk holds sa[c0 + j][seg0 + kk] at column j, sw at NT.
-// Token row of sorted row r (MoE gather), clamped into [0, T) so a malformed routing
-// table can never address outside qa / sa.
+// Token of sorted row r (MoE scatter), clamped into [0, T) so a malformed routing
+// table can never address outside the output.
 __device__ __forceinline__ int moe_token(const GemmArgs& a, int r) {
   return min(max(__ldg(a.row_token + r), 0), a.moe_T - 1);
 }
 
-template <class C, bool MOE = false>
+template <class C>
 __device__ __forceinline__ void swap_seg_load(const GemmArgs& a, const SwapSeg& s, int nbn, int nkb, uint32_t tbl,
                                               int ewarp, int lane) {
   const int cnt = min(C::NT, s.r1 - s.c0);
   const int seglen = min(C::KB_CAP, nkb - s.seg0);
-  for (int j = ewarp; j < cnt; j += kEpiThreads / 32) {
-    const int64_t row = MOE ? int64_t(moe_token(a, s.c0 + j)) : int64_t(s.c0 + j);
-    const float* src = a.sa + row * nkb + s.seg0;
+  const float* src = a.sa + int64_t(s.c0) * nkb + s.seg0;
+  for (int j = ewarp; j < cnt; j += kEpiThreads / 32)
     for (int kk = lane; kk < seglen; kk += 32)
-      cp_async4(tbl + 4u * uint32_t(kk * C::TROW + j), src + kk);
-  }
+      cp_async4(tbl + 4u * uint32_t(kk * C::TROW + j), src + int64_t(j) * nkb + kk);
   if (ewarp == 0) {
     const float* sws = a.sw + (int64_t(s.u / nbn) * nbn + s.u % nbn) * nkb + s.seg0;
     for (int kk = lane; kk < seglen; kk += 32) cp_async4(tbl + 4u * uint32_t(kk * C::TROW + C::NT), sws + kk);
@@ -159,9 +157,9 @@ __device__ __forceinline__ void swap_seg_load(const GemmArgs& a, const SwapSeg& 
 // for the next layer (dense GEMM only; args.qy / args.sy / args.qmode).  A group's 128
 // outputs sit one per thread across a warpgroup, so each warp reduces its 32 and the
 // four warps exchange maxima through shared memory under a bounded mbarrier.
-// MOE: the grouped GEMM gathers its token rows through args.row_token (tile::gather4,
-// four rows per load, from the token-major qa) and adds each output, weighted by
-// args.row_weight, into args.moe_out[token] (fp32 reductions) instead of storing y.
+// MOE: the grouped GEMM (over expert-sorted rows, as produced by act_quant_permute)
+// adds each output row r, weighted by args.row_weight[r], into
+// args.moe_out[args.row_token[r]] (fp32 reductions) instead of storing y.
 template <int NT, int NBUF, int STAGES, int KB_CAP, bool QOUT = false, bool MOE = false>
 __global__ void __launch_bounds__(kThreads, 1)
     k_gemm_swap(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
@@ -174,7 +172,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* gbase = smem_raw + (base - raw);
   float* table = reinterpret_cast<float*>(gbase + size_t(STAGES) * C::STAGE_BYTES);
   float* red = reinterpret_cast<float*>(gbase + size_t(STAGES) * C::STAGE_BYTES + 2 * size_t(C::TBUF_BYTES));
-  auto* ps = reinterpret_cast<SwapState<STAGES, NBUF>*>(gbase + size_t(STAGES) * C::STAGE_BYTES + 2 * size_t(C::TBUF_BYTES) +
+  auto* ps = reinterpret_cast<SwapState<STAGES, NBUF>*>(reinterpret_cast<uint8_t*>(red) +
                                                          (QOUT ? swap_red_bytes<C>() : 0));
   volatile int* abort = &ps->abort;
 
@@ -220,9 +218,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         group_range(args, e, r0, r1);
         for (int c0 = r0; c0 < r1 && !*abort; c0 += NT) {
           const int cnt = min(NT, r1 - c0);
-          // MOE: groups of 4 gathered rows (the last group repeats the chunk's last row)
-          const int nbox = MOE ? (cnt + 3) / 4 : (cnt + 31) / 32;
-          const uint32_t box_rows = MOE ? 4u : 32u;
+          const int nbox = (cnt + 31) / 32;
+          const uint32_t box_rows = 32u;
           for (int kb = 0; kb < nkb; ++kb, ++it) {
             const int s = it % STAGES;
             const uint32_t ph = (it / STAGES) & 1u;
@@ -231,17 +228,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t bar = smem_u32(&ps->full[s]);
             mbar_arrive_expect_tx(bar, C::W_BYTES + uint32_t(nbox) * box_rows * kTileBytesPerRow);
             tma_load_2d(w_addr, &tmW, bar, kb * kBK, e * args.N + nb * 128);
-            if constexpr (MOE) {
-              for (int i = 0; i < nbox; ++i) {
-                const int rr = c0 + 4 * i;
-                tma_gather4(w_addr + C::W_BYTES + i * 4 * kTileBytesPerRow, &tmX, bar, kb * kBK,
-                            moe_token(args, rr), moe_token(args, min(rr + 1, r1 - 1)),
-                            moe_token(args, min(rr + 2, r1 - 1)), moe_token(args, min(rr + 3, r1 - 1)));
-              }
-            } else {
-              for (int i = 0; i < nbox; ++i)
-                tma_load_2d(w_addr + C::W_BYTES + i * 32 * kTileBytesPerRow, &tmX, bar, kb * kBK, c0 + 32 * i);
-            }
+            for (int i = 0; i < nbox; ++i)
+              tma_load_2d(w_addr + C::W_BYTES + i * 32 * kTileBytesPerRow, &tmX, bar, kb * kBK, c0 + 32 * i);
           }
         }
       }
@@ -292,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t rph = 0;                    // phases of this warpgroup's exchange barrier
     SwapSeg cur;
     bool have = swap_seg_find(args, nbn, num_units, blockIdx.x, cur);
-    if (have) swap_seg_load<C, MOE>(args, cur, nbn, nkb, table_s, ewarp, lane);
+    if (have) swap_seg_load<C>(args, cur, nbn, nkb, table_s, ewarp, lane);
     uint32_t sidx = 0, sph = 0, kbc = 0;
     bool aborted = false;
     uint64_t acc[CW / 2];                                // CW fp32 accumulators as packed pairs
@@ -314,7 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       {
         SwapSeg nxt = cur;
         if (swap_seg_next<NT, KB_CAP>(args, nbn, num_units, nkb, nxt))
-          swap_seg_load<C, MOE>(args, nxt, nbn, nkb, table_s + ((sidx + 1) & 1u) * C::TBUF_BYTES, ewarp, lane);
+          swap_seg_load<C>(args, nxt, nbn, nkb, table_s + ((sidx + 1) & 1u) * C::TBUF_BYTES, ewarp, lane);
       }
       float* tb = table + (sidx & 1u) * (C::TBUF_BYTES / 4);
       // Fold sw[kb] into the segment's rows once, so the promotion multiplies by one
@@ -421,16 +409,29 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++rph;
           if (__any_sync(0xffffffffu, !rok)) { aborted = true; break; }
         }
-      } else if (MOE && cur.seg0 + seglen >= nkb && n < args.N) {
-        // weighted scatter-add of the expert outputs into the token-major result
+      } else if (MOE && cur.seg0 + seglen >= nkb) {
+        // weighted scatter-add of the expert outputs into the token-major result: the
+        // warp's columns' tokens and gate weights are loaded once (one per lane) and
+        // broadcast; each add is a fire-and-forget reduction
         const int ncols = max(0, min(CW, min(NT, cur.r1 - cur.c0) - col0));
+        constexpr int CQ = (CW + 31) / 32;
+        int tkn[CQ];
+        float gwt[CQ];
+#pragma unroll
+        for (int q = 0; q < CQ; ++q) {
+          const int jj = q * 32 + lane;
+          const int r = cur.c0 + col0 + jj;
+          tkn[q] = jj < ncols ? moe_token(args, r) : 0;
+          gwt[q] = jj < ncols ? __ldg(args.row_weight + r) : 0.0f;
+        }
 #pragma unroll
         for (int j = 0; j < CW; ++j) {
-          if (j < ncols) {
-            const int r = cur.c0 + col0 + j;
+          if (j < ncols) {                   // uniform across the warp
+            const int t = __shfl_sync(0xffffffffu, tkn[j / 32], j % 32);
+            const float g = __shfl_sync(0xffffffffu, gwt[j / 32], j % 32);
             const float2 f = unpack2(acc[j / 2]);
             const float v = (j & 1) ? f.y : f.x;
-            atomicAdd(args.moe_out + int64_t(moe_token(args, r)) * args.N + n, __fmul_rn(__ldg(args.row_weight + r), v));
+            if (n < args.N) red_add_f32(args.moe_out + int64_t(t) * args.N + n, __fmul_rn(g, v));
           }
         }
       } else if (cur.seg0 + seglen >= nkb && n < args.N) {

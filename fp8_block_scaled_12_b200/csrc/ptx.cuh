@@ -110,18 +110,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* m, 
       : "memory");
 }
 
-// Four rows of a 2-D tensor (each one box of 128 bytes x 1 row) at arbitrary row
-// coordinates r0..r3, written to 4 consecutive 128-byte rows of shared memory from
-// `dst`; completion counted on `bar`.  The tensor map's box must be one row high.
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* m, uint32_t bar, int32_t c0,
-                                            int32_t r0, int32_t r1, int32_t r2, int32_t r3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
-      : "memory");
-}
-
 // ------------------------------------------------------------------- tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
@@ -236,6 +224,11 @@ __device__ __forceinline__ void ffma2(uint64_t& acc, uint32_t p_lo, uint32_t p_h
   asm("{\n\t.reg .b64 t;\n\tmov.b64 t, {%1, %2};\n\tfma.rn.f32x2 %0, t, %3, %0;\n\t}"
       : "+l"(acc)
       : "r"(p_lo), "r"(p_hi), "l"(s2));
+}
+
+// *p += v in global memory without waiting for (or returning) the old value.
+__device__ __forceinline__ void red_add_f32(float* p, float v) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
 }
 
 // ------------------------------------------------- small asynchronous copies

@@ -163,10 +163,15 @@ __host__ __device__ __forceinline__ int64_t mx_tiled_offset(int64_t r, int64_t g
 // ue8m0 rule and is stored as its E8M0 byte (the fp32 exponent field of the power of
 // two) in s_out, in the tiled layout of mx_tiled_offset.  Otherwise s_out = fp32
 // [M][ceil(K/128)].
-template <int FMT, int SF, int UNROLL, bool MX = false>
+//
+// PERMUTE = true writes each row's codes and scales to perm_k rows of the output, row
+// m going to rows perm[m * perm_k + j] (MoE: a token's k expert-sorted rows), so the
+// grouped GEMM reads contiguous rows and the permutation costs no separate pass.
+template <int FMT, int SF, int UNROLL, bool MX = false, bool PERMUTE = false>
 __global__ void __launch_bounds__(256) k_act_quant(const uint16_t* __restrict__ x, int64_t M,
                                                    int64_t K, int64_t ldx, uint8_t* __restrict__ q,
-                                                   void* __restrict__ s_out) {
+                                                   void* __restrict__ s_out, const int32_t* __restrict__ perm = nullptr,
+                                                   int perm_k = 1, int64_t perm_rows = 0) {
   static_assert(!MX || SF == kScaleUe8m0, "MXFP8 exponents follow the ue8m0 rule");
   const int64_t ng = (K + 127) / 128;
   const int64_t total = M * ng;
@@ -207,7 +212,24 @@ __global__ void __launch_bounds__(256) k_act_quant(const uint16_t* __restrict__ 
         a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
       }
       const GroupScale<FMT, SF> sc(a);
-      if (item_ok[u]) {
+      if (PERMUTE && item_ok[u]) {
+        uint4 c[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint2 lo = quant8<FMT, SF>(v[u][2 * h], sc);
+          const uint2 hi = quant8<FMT, SF>(v[u][2 * h + 1], sc);
+          c[h] = make_uint4(lo.x, lo.y, hi.x, hi.y);
+        }
+        for (int j = 0; j < perm_k; ++j) {
+          // destination rows are clamped so a malformed permutation stays in bounds
+          const int64_t dr = min(max(int64_t(__ldg(perm + row[u] * perm_k + j)), int64_t(0)), perm_rows - 1);
+          uint8_t* dst = q + dr * K + col[u];
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            if (col[u] + 16 * h < K) *reinterpret_cast<uint4*>(dst + 16 * h) = c[h];
+          if (qt == 0) static_cast<float*>(s_out)[dr * ng + (col[u] >> 7)] = sc.s;
+        }
+      } else if (item_ok[u]) {
         uint8_t* dst = q + row[u] * K + col[u];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {

@@ -95,7 +95,7 @@ def main():
         print(f"gemm M={a.M} N={a.N} K={a.K} {a.scale} {a.out}: {ms * 1e3:.2f} us  {fl / ms / 1e9:.1f} TFLOPS  "
               f"{b / ms / 1e6:.1f} GB/s")
     elif a.op == "moe":
-        # routed layer: scores -> route, act_quant of the tokens, gather GEMM + weighted scatter
+        # routed layer: scores -> route, act_quant into sorted rows, GEMM + weighted scatter
         g = torch.Generator(device=dev).manual_seed(3)
         scores = torch.rand((a.tokens, a.E), generator=g, device=dev, dtype=torch.float32)
         x = synth.activations(a.tokens, a.K, seed=0, device=dev)
@@ -105,8 +105,9 @@ def main():
         for e in range(a.E):
             F.fp8_weight_quant(synth.weights(a.N, a.K, 0.02, seed=0, chunk=e, device=dev), qw[e], sw[e])
         route = F.moe_route(scores, a.topk)
+        qs, ss = F.act_quant_permute(x, route)
         out = torch.empty((a.tokens, a.N), dtype=torch.float32, device=dev)
-        ms = timed(lambda: F.fp8_moe_gemm(qa, sa, qw, sw, route, out), a.warm, a.iters)
+        ms = timed(lambda: F.fp8_moe_gemm(qs, ss, qw, sw, route, out), a.warm, a.iters)
         fl = 2.0 * a.tokens * a.topk * a.N * a.K
         print(f"moe_gemm tokens={a.tokens} E={a.E} top-{a.topk} N={a.N} K={a.K}: {ms * 1e3:.1f} us  "
               f"{fl / ms / 1e9:.1f} TFLOPS")

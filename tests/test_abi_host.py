@@ -226,3 +226,10 @@ def test_moe_validation():
     assert mg(FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, 16, 4, 2, 256, 256, FAKE, S) == INVALID
     assert mg(FAKE + 8, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 16, 4, 2, 256, 256, FAKE, S) == ALIGN
     assert mg(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 4, 2, 256, 256, FAKE, S) == OK
+    ap = F.lib.fp8_act_quant_permute
+    # (x, T, K, ldx, fmt, scale_fmt, token_row, k, q, s, stream)
+    assert ap(FAKE, 16, 256, 256, 0, 0, FAKE, 0, FAKE, FAKE, S) == INVALID      # k
+    assert ap(FAKE, 16, 250, 256, 0, 0, FAKE, 2, FAKE, FAKE, S) == SHAPE        # K % 16
+    assert ap(FAKE, 16, 256, 256, 0, 0, None, 2, FAKE, FAKE, S) == INVALID
+    assert ap(FAKE, 16, 256, 256, 0, 0, FAKE + 2, 2, FAKE, FAKE, S) == ALIGN
+    assert ap(FAKE, 0, 256, 256, 0, 0, None, 2, None, None, S) == OK

@@ -1,6 +1,7 @@
 """GPU parity of MoE routing (bit-exact: expert ids, gate weights, offsets and the
-sorted permutation) and of the grouped GEMM with gathered inputs and the gate-weighted
-scatter-add of its outputs, against the oracle.
+sorted permutation), of act_quant written straight into the expert-sorted rows
+(bit-exact with the oracle's act_quant of the tokens, permuted), and of the grouped
+GEMM with the gate-weighted scatter-add of its outputs fused in, against the oracle.
 
 Combine tolerance, derived: each expert output carries the block GEMM's error
 (1e-5 * sum|a w| per element, the tolerance the other GEMM tests use); the gate product
@@ -54,17 +55,24 @@ def moe_compare(dev, T, E, k, N, K, seed, tokens=None):
     scores = scores_for(T, E, seed)
     r, ro = route_both(dev, scores, k)
     x = synth.activations(T, K, seed=seed, device=dev)
-    qa, sa = F.act_quant(x)
+    qa, sa = F.act_quant(x)                      # token-major, for the oracle's combine
+    qs, ss = F.act_quant_permute(x, r)           # expert-sorted, for the GEMM
+    torch.cuda.synchronize()
+    qar, sar = O.act_quant(x.cpu(), threads=THREADS)
+    perm = np.empty(T * k, np.int64)
+    perm[ro["token_row"]] = np.repeat(np.arange(T), k)   # sorted row -> token
+    assert np.array_equal(codes(qs), qar[perm]), "permuted activation codes"
+    assert np.array_equal(ss.cpu().numpy().view(np.uint32), sar[perm].view(np.uint32)), "permuted scales"
     qw = torch.empty((E, N, K), dtype=torch.uint8, device=dev)
     sw = torch.empty((E, (N + 127) // 128, K // 128), dtype=torch.float32, device=dev)
     for e in range(E):
         F.fp8_weight_quant(synth.weights(N, K, 0.02, seed=seed, chunk=e, device=dev), qw[e], sw[e])
-    out = F.moe_gemm(qa, sa, qw, sw, r)
+    out = F.moe_gemm(qs, ss, qw, sw, r)
     torch.cuda.synchronize()
     assert F.fp8_device_error() == 0
     toks = np.arange(T) if tokens is None else np.asarray(tokens)
-    ref, bound = O.moe_combine_rows(codes(qa), sa.cpu().numpy(), codes(qw), sw.cpu().numpy(), ro["ids"], ro["w"],
-                                    toks, threads=THREADS)
+    ref, bound = O.moe_combine_rows(qar, sar, codes(qw), sw.cpu().numpy(), ro["ids"], ro["w"], toks,
+                                    threads=THREADS)
     rel = 1e-5 + (k + 1) * 2.0 ** -24
     check_fp32(out.cpu().numpy()[toks], ref, bound, f"moe T={T} E={E} k={k} N={N} K={K}", rel=rel)
 
