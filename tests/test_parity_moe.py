@@ -78,7 +78,7 @@ def moe_compare(dev, T, E, k, N, K, seed, tokens=None):
 
 
 @pytest.mark.parametrize("T,E,k,N,K", [(40, 8, 2, 256, 512), (300, 16, 4, 272, 1024), (1000, 64, 8, 1024, 384)])
-def test_moe_gemm_gather_scatter(cuda_device, T, E, k, N, K):
+def test_moe_layer_permute_scatter(cuda_device, T, E, k, N, K):
     """Ragged experts (some empty), ragged N, chunks of 160 routed rows; the last case
     has 512 units over at most 148 CTAs.  Every token."""
     moe_compare(cuda_device, T, E, k, N, K, seed=T)
