@@ -76,6 +76,27 @@ bool make_map_u8(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, 
 // ---------------------------------------------------------- GEMM launches
 constexpr int kWideStages = 4;
 
+// Every kernel is launched with programmatic stream serialisation: the runtime may
+// schedule it while the previous kernel on the stream is finishing (its prologue --
+// barrier set-up, tensor-memory allocation, descriptor and weight prefetch -- then
+// overlaps that kernel's tail), and the kernel waits for the previous one (pdl_wait)
+// before it touches operand data.  Preceding work that is not a kernel (a memset, a
+// copy) orders the launch as usual.
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 // The warpgroup register split inside the GEMM kernels (setmaxnreg) draws on the
 // registers the CTA was launched with; refuse to launch a build whose register
 // count differs from the one the split was sized for (it could never satisfy
@@ -102,8 +123,7 @@ int launch_swap(const void* qa, const void* qw, const GemmArgs& a, int64_t w_row
   const int nbn = (a.N + 127) / 128;
   const int64_t units = int64_t(a.E) * nbn;
   const int grid = int(units < num_sms() ? units : num_sms());
-  kern<<<grid, kThreads, smem, st>>>(mw, mx, a);
-  return cuda_status(cudaGetLastError());
+  return cuda_status(launch(kern, grid, kThreads, smem, st, mw, mx, a));
 }
 
 // Block-scaled (power-of-two) GEMM on the tensor core's scale path.  WIDE: P = 128
@@ -127,8 +147,7 @@ int launch_mx(const void* qa, const void* qw, const MxArgs& a, cudaStream_t st) 
   const int64_t tiles = SWAP ? int64_t((a.N + 127) / 128) * ((a.M + NQ - 1) / NQ)
                              : int64_t((a.M + 127) / 128) * ((a.N + NQ - 1) / NQ);
   const int grid = int(tiles < num_sms() ? tiles : num_sms());
-  kern<<<grid, kThreads, smem, st>>>(mp, mq, a);
-  return cuda_status(cudaGetLastError());
+  return cuda_status(launch(kern, grid, kThreads, smem, st, mp, mq, a));
 }
 
 template <bool QOUT = false>
@@ -143,8 +162,7 @@ int launch_wide(const void* qa, const void* qw, const GemmArgs& a, cudaStream_t 
   if (e != cudaSuccess) return FP8_ERR_CUDA;
   const int64_t tiles = int64_t((a.M + C::BM - 1) / C::BM) * ((a.N + C::BN - 1) / C::BN);
   const int grid = int(tiles < num_sms() ? tiles : num_sms());
-  kern<<<grid, kThreads, C::SMEM, st>>>(ma, mb, a);
-  return cuda_status(cudaGetLastError());
+  return cuda_status(launch(kern, grid, kThreads, C::SMEM, st, ma, mb, a));
 }
 
 // ------------------------------------------------------ quantiser launches
@@ -162,8 +180,8 @@ int launch_act_quant(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, uint8
   const int64_t per_warp = (steps + max_warps - 1) / max_warps;
   const int64_t warps = (steps + per_warp - 1) / per_warp;
   const int64_t blocks = (warps + 7) / 8;
-  k_act_quant<FMT, SF, U><<<int(blocks), 256, 0, st>>>(x, M, K, ldx, q, s);
-  return cuda_status(cudaGetLastError());
+  return cuda_status(launch(k_act_quant<FMT, SF, U>, unsigned(blocks), 256, 0, st, x, M, K, ldx, q, s,
+                            static_cast<const int32_t*>(nullptr), 1, int64_t(0)));
 }
 
 template <int FMT, int SF>
@@ -176,8 +194,8 @@ int launch_act_quant_permute(const uint16_t* x, int64_t M, int64_t K, int64_t ld
   const int64_t per_warp = (steps + max_warps - 1) / max_warps;
   const int64_t warps = (steps + per_warp - 1) / per_warp;
   const int64_t blocks = (warps + 7) / 8;
-  k_act_quant<FMT, SF, U, false, true><<<int(blocks), 256, 0, st>>>(x, M, K, ldx, q, s, perm, k, M * k);
-  return cuda_status(cudaGetLastError());
+  return cuda_status(launch(k_act_quant<FMT, SF, U, false, true>, unsigned(blocks), 256, 0, st, x, M, K, ldx, q, s,
+                            perm, k, M * k));
 }
 
 template <int FMT>
@@ -190,8 +208,8 @@ int launch_mx_quant(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, uint8_
   const int64_t per_warp = (steps + max_warps - 1) / max_warps;
   const int64_t warps = (steps + per_warp - 1) / per_warp;
   const int64_t blocks = (warps + 7) / 8;
-  k_act_quant<FMT, kScaleUe8m0, U, true><<<int(blocks), 256, 0, st>>>(x, M, K, ldx, q, e8);
-  return cuda_status(cudaGetLastError());
+  return cuda_status(launch(k_act_quant<FMT, kScaleUe8m0, U, true>, unsigned(blocks), 256, 0, st, x, M, K, ldx, q, e8,
+                            static_cast<const int32_t*>(nullptr), 1, int64_t(0)));
 }
 
 template <int FMT>
@@ -200,15 +218,13 @@ int launch_dequant(const uint8_t* q, const float* s, int64_t N, int64_t K, int b
   int64_t blocks = (total + 255) / 256;
   const int64_t cap = int64_t(num_sms()) * 8;
   if (blocks > cap) blocks = cap;
-  k_weight_dequant<FMT><<<int(blocks), 256, 0, st>>>(q, s, N, K, block, w);
-  return cuda_status(cudaGetLastError());
+  return cuda_status(launch(k_weight_dequant<FMT>, unsigned(blocks), 256, 0, st, q, s, N, K, block, w));
 }
 
 template <int FMT, int SF>
 int launch_block_quant(const uint16_t* w, int64_t N, int64_t K, uint8_t* q, float* s, cudaStream_t st) {
   dim3 grid(unsigned((K + 127) / 128), unsigned((N + 127) / 128));
-  k_block_quant<FMT, SF><<<grid, 256, 0, st>>>(w, N, K, q, s);
-  return cuda_status(cudaGetLastError());
+  return cuda_status(launch(k_block_quant<FMT, SF>, grid, 256, 0, st, w, N, K, q, s));
 }
 
 template <int FMT, int SF>
@@ -221,16 +237,17 @@ int launch_tensor_quant(const uint16_t* x, int64_t n, uint8_t* q, float* s, cuda
   unsigned int* slot = reinterpret_cast<unsigned int*>(s);
   cudaError_t e = cudaMemsetAsync(slot, 0, sizeof(unsigned int), st);
   if (e != cudaSuccess) return FP8_ERR_CUDA;
-  k_tensor_amax<<<int(blocks), 256, 0, st>>>(x, n8, slot);
-  k_tensor_cast<FMT, SF><<<int(blocks), 256, 0, st>>>(x, n8, slot, q);
-  k_tensor_scale<FMT, SF><<<1, 1, 0, st>>>(slot);
-  return cuda_status(cudaGetLastError());
+  if (launch(k_tensor_amax, unsigned(blocks), 256, 0, st, x, n8, slot) != cudaSuccess) return FP8_ERR_CUDA;
+  if (launch(k_tensor_cast<FMT, SF>, unsigned(blocks), 256, 0, st, x, n8, slot, q) != cudaSuccess) return FP8_ERR_CUDA;
+  return cuda_status(launch(k_tensor_scale<FMT, SF>, 1, 1, 0, st, slot));
 }
 
 // One warp whose mbarrier never completes: the bounded wait that every pipelined
 // wait of the GEMM kernels uses gives up after limit_ns, records the timeout in the
 // device error word and the kernel returns normally.
 __global__ void k_selftest_wait(uint64_t limit_ns) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ uint64_t bar;
   __shared__ int abort_flag;
   if (threadIdx.x == 0) {
@@ -408,12 +425,11 @@ int fp8_delayed_quant(const void* x, int64_t n, int fmt, float target, int64_t h
   const uint16_t* xb = static_cast<const uint16_t*>(x);
   uint8_t* qb = static_cast<uint8_t*>(q);
   unsigned long long* nc = reinterpret_cast<unsigned long long*>(n_clipped);
-  if (fmt == FP8_E4M3)
-    k_delayed_cast<kE4M3><<<int(blocks), 256, 0, st>>>(xb, n8, scale, pos, int(hist_len), history, qb, nc, s_used);
-  else
-    k_delayed_cast<kE5M2><<<int(blocks), 256, 0, st>>>(xb, n8, scale, pos, int(hist_len), history, qb, nc, s_used);
-  k_delayed_finalize<<<1, 32, 0, st>>>(target, int(hist_len), algo, scale, pos, history);
-  return cuda_status(cudaGetLastError());
+  const cudaError_t e = fmt == FP8_E4M3
+      ? launch(k_delayed_cast<kE4M3>, unsigned(blocks), 256, 0, st, xb, n8, scale, pos, int(hist_len), history, qb, nc, s_used)
+      : launch(k_delayed_cast<kE5M2>, unsigned(blocks), 256, 0, st, xb, n8, scale, pos, int(hist_len), history, qb, nc, s_used);
+  if (e != cudaSuccess) return FP8_ERR_CUDA;
+  return cuda_status(launch(k_delayed_finalize, 1, 32, 0, st, target, int(hist_len), algo, scale, pos, history));
 }
 
 int fp8_mx_quant(const void* x, int64_t M, int64_t K, int64_t ldx, int fmt, void* q, void* e8, void* stream) {
@@ -458,9 +474,8 @@ int fp8_mx_pack_pow2(const float* s, int64_t rows, int64_t K, int row_block, voi
   if (!s || !sf) return FP8_ERR_INVALID_ARG;
   if (!aligned(s, 4) || !aligned(sf, 16)) return FP8_ERR_ALIGNMENT;
   const int64_t nkb = K / 128, n = rows * nkb;
-  k_mx_pack_pow2<<<unsigned((n + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      s, rows, nkb, row_block, static_cast<uint8_t*>(sf));
-  return cuda_status(cudaGetLastError());
+  return cuda_status(launch(k_mx_pack_pow2, unsigned((n + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream), s, rows,
+                            nkb, row_block, static_cast<uint8_t*>(sf)));
 }
 
 int fp8_moe_route(const float* scores, int64_t T, int64_t E, int64_t k, int32_t* ids, float* w, int32_t* offsets,
@@ -475,17 +490,15 @@ int fp8_moe_route(const float* scores, int64_t T, int64_t E, int64_t k, int32_t*
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (T > 0) {
     const int blocks = int((T * 32 + 255) / 256);
-    if (E <= 256)
-      k_moe_topk<8><<<blocks, 256, 0, st>>>(scores, int(T), int(E), int(k), ids, w);
-    else
-      k_moe_topk<32><<<blocks, 256, 0, st>>>(scores, int(T), int(E), int(k), ids, w);
-    if (cudaGetLastError() != cudaSuccess) return FP8_ERR_CUDA;
+    const cudaError_t e = E <= 256 ? launch(k_moe_topk<8>, unsigned(blocks), 256, 0, st, scores, int(T), int(E), int(k), ids, w)
+                                   : launch(k_moe_topk<32>, unsigned(blocks), 256, 0, st, scores, int(T), int(E), int(k), ids, w);
+    if (e != cudaSuccess) return FP8_ERR_CUDA;
   }
   const size_t smem = size_t(32) * size_t(E) * sizeof(int32_t);
   if (cudaFuncSetAttribute(k_moe_sort, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
     return FP8_ERR_CUDA;
-  k_moe_sort<<<1, 1024, smem, st>>>(ids, w, int(T), int(E), int(k), offsets, row_token, row_weight, token_row);
-  return cuda_status(cudaGetLastError());
+  return cuda_status(launch(k_moe_sort, 1, 1024, smem, st, static_cast<const int32_t*>(ids), static_cast<const float*>(w),
+                            int(T), int(E), int(k), offsets, row_token, row_weight, token_row));
 }
 
 int fp8_act_quant_permute(const void* x, int64_t T, int64_t K, int64_t ldx, int fmt, int scale_fmt,
@@ -534,8 +547,7 @@ int fp8_moe_gemm(const void* qa, const float* sa, const void* qw, const float* s
 
 int fp8_selftest_bounded_wait(int64_t limit_ns, void* stream) {
   if (limit_ns <= 0 || limit_ns > 10000000000ll) return FP8_ERR_INVALID_ARG;
-  k_selftest_wait<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(uint64_t(limit_ns));
-  return cuda_status(cudaGetLastError());
+  return cuda_status(launch(k_selftest_wait, 1, 32, 0, static_cast<cudaStream_t>(stream), uint64_t(limit_ns)));
 }
 
 int fp8_device_error(void* stream) {

@@ -148,6 +148,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_barrier_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (int(blockIdx.x) < num_tiles)     // first weight tiles of the first tile, to L2
+      for (int kb = 0; kb < STAGES && kb < nkb; ++kb)
+        tma_prefetch_l2_2d(&tmB, kb * kBK, (int(blockIdx.x) / num_m) * C::BN);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(&ps->tmem_base), C::TMEM_COLS);
@@ -156,6 +159,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_wait();
   const uint32_t tmem = ps->tmem_base;
 
   if (warp < 4) {
@@ -176,6 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(sa_ + C::A_BYTES, &tmB, bar, kb * kBK, nb * C::BN);
         }
       }
+      pdl_trigger();                     // every load of this CTA is issued
     } else if (warp == 1 && lane == 0) {
       // ------------------------------------------------ MMA issuer
       constexpr uint32_t idesc = idesc_f8_e4m3_f32(C::BM, C::BN);

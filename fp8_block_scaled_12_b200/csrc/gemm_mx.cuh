@@ -203,6 +203,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_barrier_init();
     tma_prefetch_desc(&tmP);
     tma_prefetch_desc(&tmQ);
+    if (int(blockIdx.x) < num_tiles) {   // first weight tiles of the first tile, to L2
+      int p0, q0, qn;
+      mx_tile<C>(args, blockIdx.x, p0, q0, qn);
+      for (int kb = 0; kb < C::STAGES && kb < nkb; ++kb) {
+        if (C::SWAP)
+          tma_prefetch_l2_2d(&tmP, kb * kBK, p0);
+        else
+          tma_prefetch_l2_2d(&tmQ, kb * kBK, q0);
+      }
+    }
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(&ps->tmem_base), C::TMEM_COLS);
@@ -211,6 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_wait();
   const uint32_t tmem = ps->tmem_base;
 
   if (warp < 4) {
@@ -247,6 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             bulk_load(sfs + 512u * (1 + a), sfq + (size_t(qa0 + a) * nkb + kb) * 512, 512u, bar);
         }
       }
+      pdl_trigger();                     // every load of this CTA is issued
     } else if (warp == 1 && lane == 0) {
       // ------------------------------------------------ MMA issuer
       uint32_t it = 0, tc = 0;
@@ -360,6 +372,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 // scale that is not a positive normal power of two raises kErrBadScale.
 __global__ void __launch_bounds__(256) k_mx_pack_pow2(const float* __restrict__ s, int64_t rows, int64_t nkb,
                                                       int row_block, uint8_t* __restrict__ out) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= rows * nkb) return;
   const int64_t r = i / nkb, kb = i - r * nkb;

@@ -197,6 +197,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_barrier_init();
     tma_prefetch_desc(&tmW);
     tma_prefetch_desc(&tmX);
+    // the first weight tiles of this CTA's first unit go to L2 while the previous
+    // kernel finishes (an empty expert's prefetch is only a wasted hint)
+    if (int(blockIdx.x) < num_units) {
+      const int e0 = blockIdx.x / nbn, nb0 = blockIdx.x % nbn;
+      for (int kb = 0; kb < STAGES && kb < nkb; ++kb) tma_prefetch_l2_2d(&tmW, kb * kBK, e0 * args.N + nb0 * 128);
+    }
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(&ps->tmem_base), C::TMEM_COLS);
@@ -206,6 +212,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ps->tmem_base;
+  pdl_wait();
 
   if (warp < 4) {
     setmaxnreg_dec<kProducerRegs>();
@@ -233,6 +240,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      pdl_trigger();                     // every load of this CTA is issued
     } else if (warp >= 1 && warp <= kSwapIssuers && lane == 0) {
       // ------------------------------------------------ MMA issuers (round robin over K-blocks)
       const uint32_t mine = uint32_t(warp - 1);

@@ -15,6 +15,8 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include "ptx.cuh"
+
 namespace fp8lin {
 
 constexpr int kMoeMaxE = 1024;     // experts (scores per token kept in registers: 32 per lane)
@@ -23,6 +25,8 @@ constexpr int kMoeMaxK = 32;       // experts per token
 template <int EPL>
 __global__ void __launch_bounds__(256) k_moe_topk(const float* __restrict__ scores, int T, int E, int k,
                                                   int32_t* __restrict__ ids, float* __restrict__ w) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (t >= T) return;
@@ -76,6 +80,8 @@ __global__ void __launch_bounds__(1024) k_moe_sort(const int32_t* __restrict__ i
                                                    int T, int E, int k, int32_t* __restrict__ offsets,
                                                    int32_t* __restrict__ row_token, float* __restrict__ row_weight,
                                                    int32_t* __restrict__ token_row) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ int32_t cnt[];    // [32][E]: per-warp counts, then per-warp first slots
   __shared__ int32_t tot[kMoeMaxE];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;

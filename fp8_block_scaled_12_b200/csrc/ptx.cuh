@@ -98,6 +98,25 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
 }
 
+// L2 prefetch of one 2-D tile through a tensor map (no shared memory, no completion).
+// The L2 is the point of coherence for device memory, so a prefetch issued before the
+// grid-dependency wait can never hand stale data to a later load.
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* m, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(m)),
+               "r"(x), "r"(y)
+               : "memory");
+}
+
+// Programmatic dependent launch.  Every kernel of the library is launched so that it
+// may start while the previous kernel on the stream is finishing; pdl_wait() blocks
+// the calling thread until that kernel has completed and its writes are visible, so
+// each kernel calls it before its first global read or write of operand data.
+// pdl_trigger() lets the next kernel be scheduled once every CTA of this grid has
+// called it (or exited); a CTA that has not started cannot have called it, so the
+// next grid never takes SMs this grid still needs.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // 2-D tiled bulk tensor load global -> shared, completion counted on `bar`.
 // c0 is the innermost (contiguous) coordinate in elements; it must be a multiple
 // of 16 for 1-byte elements (callers only pass multiples of 128).

@@ -25,6 +25,8 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include "ptx.cuh"
+
 namespace fp8lin {
 
 enum : int { kE4M3 = 0, kE5M2 = 1 };
@@ -172,6 +174,8 @@ __global__ void __launch_bounds__(256) k_act_quant(const uint16_t* __restrict__ 
                                                    int64_t K, int64_t ldx, uint8_t* __restrict__ q,
                                                    void* __restrict__ s_out, const int32_t* __restrict__ perm = nullptr,
                                                    int perm_k = 1, int64_t perm_rows = 0) {
+  pdl_wait();
+  pdl_trigger();
   static_assert(!MX || SF == kScaleUe8m0, "MXFP8 exponents follow the ue8m0 rule");
   const int64_t ng = (K + 127) / 128;
   const int64_t total = M * ng;
@@ -259,6 +263,8 @@ template <int FMT, int SF>
 __global__ void __launch_bounds__(256) k_block_quant(const uint16_t* __restrict__ w, int64_t N,
                                                      int64_t K, uint8_t* __restrict__ q,
                                                      float* __restrict__ s_inv) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float red[8];
   const int64_t nbk = (K + 127) / 128;
   const int64_t bn = blockIdx.y, bk = blockIdx.x;
@@ -295,6 +301,8 @@ __global__ void __launch_bounds__(256) k_block_quant(const uint16_t* __restrict_
 // like their bit patterns, so an unsigned atomicMax is an exact float max).
 __global__ void __launch_bounds__(256) k_tensor_amax(const uint16_t* __restrict__ x, int64_t n8,
                                                      unsigned int* amax_bits) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float red[8];
   float a = 0.0f;
   const uint4* p = reinterpret_cast<const uint4*>(x);
@@ -325,6 +333,8 @@ template <int FMT, int SF>
 __global__ void __launch_bounds__(256) k_tensor_cast(const uint16_t* __restrict__ x, int64_t n8,
                                                      const unsigned int* amax_bits,
                                                      uint8_t* __restrict__ q) {
+  pdl_wait();
+  pdl_trigger();
   const GroupScale<FMT, SF> sc(__uint_as_float(*amax_bits));
   const uint4* p = reinterpret_cast<const uint4*>(x);
   uint2* o = reinterpret_cast<uint2*>(q);
@@ -346,6 +356,8 @@ __global__ void __launch_bounds__(256) k_tensor_cast(const uint16_t* __restrict_
 // Pass 3: replace the amax bits with the scale.
 template <int FMT, int SF>
 __global__ void k_tensor_scale(unsigned int* slot) {
+  pdl_wait();
+  pdl_trigger();
   const GroupScale<FMT, SF> sc(__uint_as_float(*slot));
   *reinterpret_cast<float*>(slot) = sc.s;
 }
@@ -407,6 +419,8 @@ __global__ void __launch_bounds__(256) k_delayed_cast(const uint16_t* __restrict
                                                       const int32_t* __restrict__ pos, int hist_len, float* history,
                                                       uint8_t* __restrict__ q, unsigned long long* n_clipped,
                                                       float* s_used) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float red_a[8];
   __shared__ uint32_t red_c[8];
   const float s = *scale;
@@ -458,6 +472,8 @@ __global__ void __launch_bounds__(256) k_delayed_cast(const uint16_t* __restrict
 // least 2^-126; then clear the next slot and advance the slot index.
 __global__ void k_delayed_finalize(float target, int hist_len, int algo, float* scale, int32_t* pos,
                                    float* history) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x;
   const int p = delayed_slot(pos, hist_len);
   float a = 0.0f;
@@ -503,6 +519,8 @@ template <int FMT>
 __global__ void __launch_bounds__(256) k_weight_dequant(const uint8_t* __restrict__ q, const float* __restrict__ s_inv,
                                                         int64_t N, int64_t K, int block,
                                                         uint16_t* __restrict__ w) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t k16 = K / 16, total = N * k16;
   const int64_t nbk = block > 0 ? (K + block - 1) / block : 1;
   const int64_t stride = int64_t(gridDim.x) * blockDim.x;
