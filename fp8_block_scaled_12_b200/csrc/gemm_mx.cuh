@@ -29,6 +29,11 @@
 //                (NQ rows) with their scale atoms into a ring of stages.
 //   warp 1       MMA issuer: per K-block, tcgen05.cp of the atoms into one of two
 //                tensor-memory scale slots, then 4 block-scaled MMAs (K = 32 each).
+//   warp 2       SWAP tiles only: a second issuer.  Issuing a K-block's copies and MMAs
+//                keeps one thread busy ~440 clk, about the whole K-block period of a
+//                weight stream, so the two issuers take alternate K-blocks, each into
+//                its own accumulator and scale slots; the epilogue adds the two
+//                accumulators (a fixed order, so the result is deterministic).
 //   warps 4-11   epilogue: after a tile's last K-block, tensor memory -> registers,
 //                release the accumulator, then convert and store while the next tile's
 //                MMAs run.
@@ -113,9 +118,10 @@ struct MxCfg {
   static constexpr uint32_t Q_BYTES = NQ * kTileBytesPerRow;
   static constexpr uint32_t STAGE_BYTES = P_BYTES + Q_BYTES;
   static constexpr uint32_t SF_BYTES = 512u * (1 + QATOMS);       // scale atoms of one stage
+  static constexpr int ISSUERS = SWAP ? 2 : 1;                    // MMA issuers, one accumulator each
   static constexpr uint32_t SF_SLOT_COLS = 16;                    // tensor-memory columns per slot
-  static constexpr uint32_t SF_COL0 = NQ;                         // after the accumulator
-  static constexpr uint32_t TMEM_NEED = NQ + 2 * SF_SLOT_COLS;
+  static constexpr uint32_t SF_COL0 = ISSUERS * NQ;               // after the accumulators
+  static constexpr uint32_t TMEM_NEED = ISSUERS * NQ + 2 * ISSUERS * SF_SLOT_COLS;
   static constexpr uint32_t TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128
                                         : TMEM_NEED <= 256 ? 256 : 512;
   static_assert(NQ % 32 == 0 && NQ >= 32 && NQ <= 256, "MMA N");
@@ -197,7 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&ps->full[s]), 1);
       mbar_init(smem_u32(&ps->empty[s]), 1);
     }
-    mbar_init(smem_u32(&ps->tfull), 1);
+    mbar_init(smem_u32(&ps->tfull), C::ISSUERS);
     mbar_init(smem_u32(&ps->tempty), kEpiThreads / 32);
     ps->abort = 0;
     fence_barrier_init();
@@ -259,9 +265,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       pdl_trigger();                     // every load of this CTA is issued
-    } else if (warp == 1 && lane == 0) {
-      // ------------------------------------------------ MMA issuer
-      uint32_t it = 0, tc = 0;
+    } else if (warp >= 1 && warp <= C::ISSUERS && lane == 0) {
+      // ------------------------------------------------ MMA issuer(s): issuer i takes the
+      // K-blocks kb % ISSUERS == i of every tile into accumulator i
+      const int mine = warp - 1;
+      const uint32_t dacc = tmem + uint32_t(mine) * C::NQ;
+      uint32_t it = 0, tc = 0, own = 0;
       bool stop = false;
       for (int t = blockIdx.x; t < num_tiles && !stop; t += gridDim.x, ++tc) {
         int p0, q0, qn;
@@ -272,10 +281,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(smem_u32(&ps->tempty), (tc & 1u) ^ 1u, abort)) break;
         tc_fence_after();
         for (int kb = 0; kb < nkb; ++kb, ++it) {
+          if (kb % C::ISSUERS != mine) continue;
           const int s = it % C::STAGES;
           if (!mbar_wait(smem_u32(&ps->full[s]), (it / C::STAGES) & 1u, abort)) { stop = true; break; }
           tc_fence_after();
-          const uint32_t slot = C::SF_COL0 + (it & 1u) * C::SF_SLOT_COLS;
+          const uint32_t slot = C::SF_COL0 + (uint32_t(mine) * 2 + (own++ & 1u)) * C::SF_SLOT_COLS;
           const uint32_t sfs = sf_base + s * C::SF_BYTES;
           tmem_cp_32x128b_x4(tmem + slot, sf_atom_desc(sfs));                          // P scales
 #pragma unroll
@@ -286,14 +296,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int k = 0; k < kBK / 32; ++k) {
             const uint32_t sfid = uint32_t(k) << 30;
-            mma_mx(tmem, sw128_kmajor_desc(pa + k * 32), sw128_kmajor_desc(qa + k * 32),
+            mma_mx(dacc, sw128_kmajor_desc(pa + k * 32), sw128_kmajor_desc(qa + k * 32),
                    idesc_mx_e4m3(128, n_mma, uint32_t(k)), (tmem + slot) | sfid, (tmem + slot + 8 + qcol) | sfid,
-                   (kb > 0 || k > 0) ? 1u : 0u);
+                   (kb >= C::ISSUERS || k > 0) ? 1u : 0u);
           }
           mma_commit(smem_u32(&ps->empty[s]));
         }
         if (stop) break;
-        mma_commit(smem_u32(&ps->tfull));
+        mma_commit(smem_u32(&ps->tfull));      // also when this issuer had no K-block (nkb == 1)
       }
     }
   } else {
@@ -318,6 +328,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       if constexpr (CW % 32 == 16) tmem_ld16(taddr + (CW - 16), *reinterpret_cast<uint32_t(*)[16]>(&v[CW - 16]));
       tmem_ld_wait();
       tmem_regs_ready(v);
+      if (C::ISSUERS == 2 && nkb > 1) {
+        // y = fl32(acc0 + acc1): the second issuer's accumulator, 16 columns at a time
+#pragma unroll
+        for (int c = 0; c < CW; c += 16) {
+          uint32_t u[16];
+          tmem_ld16(taddr + C::NQ + c, u);
+          tmem_ld_wait();
+          tmem_regs_ready(u);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[c + i] = __float_as_uint(__fadd_rn(__uint_as_float(v[c + i]), __uint_as_float(u[i])));
+        }
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&ps->tempty));
