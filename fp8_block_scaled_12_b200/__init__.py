@@ -24,7 +24,7 @@ __all__ = [
     "fp8_mx_pack_pow2", "fp8_delayed_quant", "DelayedScaling", "AMAX_MOST_RECENT", "AMAX_MAX",
     "fp8_block_gemm_quant", "fp8_weight_dequant", "block_gemm_quant", "weight_dequant",
     "fp8_moe_route", "fp8_moe_gemm", "fp8_act_quant_permute", "moe_route", "moe_gemm", "act_quant_permute",
-    "fp8_status_string", "fp8_device_error", "fp8_selftest_bounded_wait",
+    "fp8_status_string", "fp8_device_error", "fp8_selftest_bounded_wait", "fp8_set_wait_limit_ns",
     "act_quant", "weight_quant", "block_gemm", "grouped_gemm", "mx_quant", "mx_gemm", "mx_pack_pow2",
     "mx_sf_bytes", "EXPORTS",
 ]
@@ -41,7 +41,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfp8lin.s
 EXPORTS = ("fp8_act_quant", "fp8_weight_quant", "fp8_block_gemm", "fp8_grouped_gemm", "fp8_mx_quant",
            "fp8_mx_gemm", "fp8_mx_pack_pow2", "fp8_delayed_quant", "fp8_block_gemm_quant", "fp8_weight_dequant",
            "fp8_moe_route", "fp8_moe_gemm", "fp8_act_quant_permute", "fp8_status_string", "fp8_device_error",
-           "fp8_selftest_bounded_wait")
+           "fp8_selftest_bounded_wait", "fp8_set_wait_limit_ns")
 
 
 class Fp8Error(RuntimeError):
@@ -72,10 +72,11 @@ def _load() -> ctypes.CDLL:
     L.fp8_status_string.restype = ctypes.c_char_p
     L.fp8_device_error.argtypes = [vp]
     L.fp8_selftest_bounded_wait.argtypes = [i64, vp]
+    L.fp8_set_wait_limit_ns.argtypes = [i64]
     for name in ("fp8_act_quant", "fp8_weight_quant", "fp8_block_gemm", "fp8_grouped_gemm", "fp8_mx_quant",
                  "fp8_mx_gemm", "fp8_mx_pack_pow2", "fp8_delayed_quant", "fp8_block_gemm_quant",
                  "fp8_weight_dequant", "fp8_moe_route", "fp8_moe_gemm", "fp8_act_quant_permute",
-                 "fp8_device_error", "fp8_selftest_bounded_wait"):
+                 "fp8_device_error", "fp8_selftest_bounded_wait", "fp8_set_wait_limit_ns"):
         getattr(L, name).restype = ci
     return L
 
@@ -388,6 +389,11 @@ def fp8_selftest_bounded_wait(limit_ns: int, stream=None) -> None:
     """Launch the diagnostic kernel whose bounded mbarrier wait runs out after
     `limit_ns`; a following fp8_device_error() reports the timeout."""
     _check("fp8_selftest_bounded_wait", lib.fp8_selftest_bounded_wait(int(limit_ns), _stream(stream)))
+
+
+def fp8_set_wait_limit_ns(limit_ns: int) -> None:
+    """Diagnostic: limit of the GEMM kernels' bounded waits (0 restores the default)."""
+    _check("fp8_set_wait_limit_ns", lib.fp8_set_wait_limit_ns(int(limit_ns)))
 
 
 # ------------------------------------------------- allocating wrappers

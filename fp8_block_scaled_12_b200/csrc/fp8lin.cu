@@ -550,6 +550,12 @@ int fp8_selftest_bounded_wait(int64_t limit_ns, void* stream) {
   return cuda_status(launch(k_selftest_wait, 1, 32, 0, static_cast<cudaStream_t>(stream), uint64_t(limit_ns)));
 }
 
+int fp8_set_wait_limit_ns(int64_t limit_ns) {
+  if (limit_ns < 0 || limit_ns > 10000000000ll) return FP8_ERR_INVALID_ARG;
+  const unsigned long long v = limit_ns == 0 ? FP8LIN_WAIT_NS : (unsigned long long)limit_ns;
+  return cuda_status(cudaMemcpyToSymbol(g_wait_limit_ns, &v, sizeof(v)));
+}
+
 int fp8_device_error(void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(st) != cudaSuccess) return FP8_ERR_CUDA;

@@ -78,6 +78,7 @@ struct alignas(8) PipeState {
   uint64_t empty[STAGES];
   uint64_t tfull[2];
   uint64_t tempty[2];
+  uint64_t drain;          // abort path: the issuer's MMAs have finished
   uint32_t tmem_base;
   int abort;
 };
@@ -144,6 +145,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&ps->tfull[b]), 1);
       mbar_init(smem_u32(&ps->tempty[b]), kEpiThreads / 32);
     }
+    mbar_init(smem_u32(&ps->drain), 1);
     ps->abort = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmA);
@@ -180,6 +182,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(sa_ + C::A_BYTES, &tmB, bar, kb * kBK, nb * C::BN);
         }
       }
+      if (*abort) {                      // every load already issued lands before the CTA exits
+        for (uint32_t j = it > uint32_t(STAGES) ? it - uint32_t(STAGES) : 0u; j < it; ++j)
+          mbar_drain(smem_u32(&ps->full[j % STAGES]), (j / STAGES) & 1u);
+      }
       pdl_trigger();                     // every load of this CTA is issued
     } else if (warp == 1 && lane == 0) {
       // ------------------------------------------------ MMA issuer
@@ -204,6 +210,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_commit(smem_u32(&ps->empty[s]));
           mma_commit(smem_u32(&ps->tfull[b]));
         }
+      }
+      if (*abort) {                      // the MMAs already issued finish before tensor memory is freed
+        mma_commit(smem_u32(&ps->drain));
+        mbar_drain(smem_u32(&ps->drain), 0u);
       }
     }
   } else {
@@ -295,10 +305,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (*abort) {
-    if (threadIdx.x == 0) settle_ns(200000);
-    __syncthreads();
-  }
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);

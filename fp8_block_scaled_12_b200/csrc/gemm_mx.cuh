@@ -138,6 +138,7 @@ struct alignas(8) MxState {
   uint64_t empty[STAGES];
   uint64_t tfull;
   uint64_t tempty;
+  uint64_t drain[2];       // abort path: each issuer's MMAs and scale copies have finished
   uint32_t tmem_base;
   int abort;
 };
@@ -205,6 +206,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(smem_u32(&ps->tfull), C::ISSUERS);
     mbar_init(smem_u32(&ps->tempty), kEpiThreads / 32);
+    mbar_init(smem_u32(&ps->drain[0]), 1);
+    mbar_init(smem_u32(&ps->drain[1]), 1);
     ps->abort = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmP);
@@ -264,6 +267,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             bulk_load(sfs + 512u * (1 + a), sfq + (size_t(qa0 + a) * nkb + kb) * 512, 512u, bar);
         }
       }
+      if (*abort) {                      // every load already issued lands before the CTA exits
+        for (uint32_t j = it > uint32_t(C::STAGES) ? it - uint32_t(C::STAGES) : 0u; j < it; ++j)
+          mbar_drain(smem_u32(&ps->full[j % C::STAGES]), (j / C::STAGES) & 1u);
+      }
       pdl_trigger();                     // every load of this CTA is issued
     } else if (warp >= 1 && warp <= C::ISSUERS && lane == 0) {
       // ------------------------------------------------ MMA issuer(s): issuer i takes the
@@ -304,6 +311,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (stop) break;
         mma_commit(smem_u32(&ps->tfull));      // also when this issuer had no K-block (nkb == 1)
+      }
+      if (*abort) {                      // the MMAs already issued finish before tensor memory is freed
+        mma_commit(smem_u32(&ps->drain[mine]));
+        mbar_drain(smem_u32(&ps->drain[mine]), 0u);
       }
     }
   } else {
@@ -377,10 +388,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (*abort) {
-    if (threadIdx.x == 0) settle_ns(200000);
-    __syncthreads();
-  }
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);

@@ -58,6 +58,8 @@ struct SwapCfg {
   static_assert(TBUF_BYTES % 16 == 0, "table rows keep 16-byte alignment");
 };
 
+constexpr int kSwapIssuersMax = 3;
+
 template <int STAGES, int NBUF>
 struct alignas(8) SwapState {
   uint64_t full[STAGES];
@@ -66,6 +68,7 @@ struct alignas(8) SwapState {
   uint64_t tempty[NBUF];
   uint64_t seg;            // epilogue warps: segment's table loaded, previous one retired
   uint64_t red[2];         // fused output quantisation: per warpgroup, group maxima exchanged
+  uint64_t drain[kSwapIssuersMax];   // abort path: each issuer's MMAs have finished
   uint32_t tmem_base;
   int abort;
 };
@@ -97,7 +100,7 @@ __device__ __forceinline__ void group_range(const GemmArgs& a, int e, int& r0, i
   }
 }
 
-constexpr int kSwapIssuers = 3;
+constexpr int kSwapIssuers = kSwapIssuersMax;
 
 // One segment of a CTA's work: unit u (expert e = u / nbn, weight row-block
 // nb = u % nbn), token rows [c0, min(c0 + NT, r1)), K-blocks [seg0, seg0 + KB_CAP).
@@ -193,6 +196,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(smem_u32(&ps->seg), kEpiThreads / 32);
     mbar_init(smem_u32(&ps->red[0]), 4);
     mbar_init(smem_u32(&ps->red[1]), 4);
+    for (int i = 0; i < kSwapIssuers; ++i) mbar_init(smem_u32(&ps->drain[i]), 1);
     ps->abort = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmW);
@@ -240,6 +244,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      if (*abort) {                      // every load already issued lands before the CTA exits
+        for (uint32_t j = it > uint32_t(STAGES) ? it - uint32_t(STAGES) : 0u; j < it; ++j)
+          mbar_drain(smem_u32(&ps->full[j % STAGES]), (j / STAGES) & 1u);
+      }
       pdl_trigger();                     // every load of this CTA is issued
     } else if (warp >= 1 && warp <= kSwapIssuers && lane == 0) {
       // ------------------------------------------------ MMA issuers (round robin over K-blocks)
@@ -272,6 +280,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_commit(smem_u32(&ps->tfull[b]));
           }
         }
+      }
+      if (*abort) {                      // the MMAs already issued finish before tensor memory is freed
+        mma_commit(smem_u32(&ps->drain[mine]));
+        mbar_drain(smem_u32(&ps->drain[mine]), 0u);
       }
     }
   } else {
@@ -466,10 +478,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (*abort) {
-    if (threadIdx.x == 0) settle_ns(200000);
-    __syncthreads();
-  }
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);

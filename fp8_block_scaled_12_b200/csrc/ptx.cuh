@@ -24,6 +24,9 @@ namespace fp8lin {
 // a bounded wait ran out.  Read and cleared by fp8_device_error().  The whole
 // library is one translation unit, so this definition is the only one.
 __device__ unsigned int g_device_error;
+// Limit of the pipeline waits in ns (FP8LIN_WAIT_NS unless a diagnostic call lowers it
+// to exercise the timeout and abort path).
+__device__ unsigned long long g_wait_limit_ns = FP8LIN_WAIT_NS;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -68,11 +71,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Wait until the phase with the given parity of `bar` has completed.  Returns
 // false (and raises *abort) when the wait runs out or another thread of the CTA
 // has already aborted.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
-                                          uint64_t limit_ns = FP8LIN_WAIT_NS) {
+// One failed try_wait already suspends the thread for a hardware-defined time, so a
+// limit under 1 us gives up at the first poll that fails.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort, uint64_t limit_ns = 0) {
   if (mbar_try_wait(bar, parity)) return true;
+  if (limit_ns == 0) limit_ns = *reinterpret_cast<volatile unsigned long long*>(&g_wait_limit_ns);
   const uint64_t t0 = globaltimer_ns();
-  for (uint32_t i = 1; i < FP8LIN_WAIT_ITERS; ++i) {
+  for (uint32_t i = limit_ns < 1000 ? FP8LIN_WAIT_ITERS : 1u; i < FP8LIN_WAIT_ITERS; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 31u) == 0) {
       if (*abort) return false;
@@ -84,13 +89,25 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   return false;
 }
 
-// Spin for roughly `ns` nanoseconds (bounded by an iteration cap as well); used on
-// the abort path so asynchronous copies and MMAs already issued can land before
-// the CTA releases tensor memory and exits.
+// Spin for roughly `ns` nanoseconds (bounded by an iteration cap as well).
 __device__ __forceinline__ void settle_ns(uint64_t ns) {
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 0; i < (1u << 22); ++i)
     if (globaltimer_ns() - t0 > ns) break;
+}
+
+// Abort path: wait for a phase that completes on its own -- an issued TMA or bulk copy
+// landing, issued MMAs finishing -- so nothing asynchronous still writes this CTA's
+// shared or tensor memory when it releases them and exits.  Ignores the abort flag
+// and always uses the full FP8LIN_WAIT_NS; should even this run out, the thread
+// settles for a further 200 us instead.
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 0; i < FP8LIN_WAIT_ITERS; ++i) {
+    if (mbar_try_wait(bar, parity)) return;
+    if ((i & 31u) == 31u && globaltimer_ns() - t0 > FP8LIN_WAIT_NS) break;
+  }
+  settle_ns(200000);
 }
 
 // ----------------------------------------------------------------------- TMA

@@ -331,6 +331,19 @@ int fp8_device_error(void* stream);
  */
 int fp8_selftest_bounded_wait(int64_t limit_ns, void* stream);
 
+/*
+ * fp8_set_wait_limit_ns -- diagnostic with no counterpart in the pages.  Sets the
+ * limit of the bounded pipeline waits of the GEMM kernels on the current device to
+ * `limit_ns` nanoseconds (0 restores the default of 2 s; 0 <= limit_ns <= 1e10, else
+ * FP8_ERR_INVALID_ARG).  A limit under 1000 ns makes a GEMM give up at its first
+ * wait whose first poll fails: the CTA raises its abort flag, every role leaves its loop,
+ * the producer waits for the loads it has issued and each MMA issuer for its MMAs,
+ * then tensor memory is freed and the kernel returns; fp8_device_error() then reports
+ * FP8_ERR_TIMEOUT and the outputs of that call are unspecified.  Synchronous with
+ * respect to the host; affects launches made after it returns.
+ */
+int fp8_set_wait_limit_ns(int64_t limit_ns);
+
 #ifdef __cplusplus
 }
 #endif

@@ -5,8 +5,16 @@ when it runs out the kernel records FP8_ERR_TIMEOUT in a device-side error word 
 returns instead of hanging.  The diagnostic entry point runs that same wait on a
 barrier nothing ever arrives on, with a short limit, so the path is exercised here:
 the status reaches the host, is cleared by reading it, and the context keeps
-working.  Host-side failures (bad arguments) are covered by test_abi_host.py.
+working.  A second diagnostic lowers the GEMM kernels' own wait limit to 1 ns so that
+every GEMM kernel takes its abort path (drain the loads and MMAs in flight, free
+tensor memory, return) -- run in a child process, then compared bit for bit with the
+same calls at the normal limit.  Host-side failures (bad arguments) are covered by
+test_abi_host.py.
 """
+import os
+import subprocess
+import sys
+
 import pytest
 import torch
 
@@ -22,6 +30,15 @@ def test_selftest_rejects_bad_limits():
     assert F.lib.fp8_selftest_bounded_wait(0, None) == 1
     assert F.lib.fp8_selftest_bounded_wait(-5, None) == 1
     assert F.lib.fp8_selftest_bounded_wait(20_000_000_000, None) == 1
+    assert F.lib.fp8_set_wait_limit_ns(-1) == 1
+    assert F.lib.fp8_set_wait_limit_ns(20_000_000_000) == 1
+
+
+@pytest.mark.gpu
+def test_gemm_abort_path_drains_and_recovers(cuda_device):
+    child = os.path.join(os.path.dirname(os.path.abspath(__file__)), "abort_child.py")
+    r = subprocess.run([sys.executable, child], capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0 and r.stdout.strip().endswith("OK"), r.stdout[-2000:] + r.stderr[-4000:]
 
 
 @pytest.mark.gpu
