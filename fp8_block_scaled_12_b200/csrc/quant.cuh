@@ -524,22 +524,40 @@ __global__ void __launch_bounds__(256) k_weight_dequant(const uint8_t* __restric
   const int64_t k16 = K / 16, total = N * k16;
   const int64_t nbk = block > 0 ? (K + block - 1) / block : 1;
   const int64_t stride = int64_t(gridDim.x) * blockDim.x;
-  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
-    const int64_t n = i / k16, k = (i - n * k16) * 16;
-    const float s = block > 0 ? __ldg(s_inv + (n / block) * nbk + k / block) : __ldg(s_inv);
-    const uint4 c = ldg_stream(reinterpret_cast<const uint4*>(q + n * K + k));
-    const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
-    uint32_t o[8];
+  // four 16-code chunks per thread and step, all loads issued before any conversion, so
+  // each thread keeps 64 bytes of codes in flight behind the (twice larger) store stream
+  constexpr int U = 4;
+  for (int64_t i0 = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i0 < total; i0 += U * stride) {
+    uint4 c[U];
+    float s[U];
+    int64_t off[U];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float2 a = fp8x2_to_f32<FMT>(uint16_t(cw[j] & 0xFFFFu));
-      const float2 b = fp8x2_to_f32<FMT>(uint16_t(cw[j] >> 16));
-      o[2 * j] = bf16x2_rn(__fmul_rn(a.x, s), __fmul_rn(a.y, s));
-      o[2 * j + 1] = bf16x2_rn(__fmul_rn(b.x, s), __fmul_rn(b.y, s));
+    for (int u = 0; u < U; ++u) {
+      const int64_t i = i0 + u * stride;
+      off[u] = -1;
+      if (i < total) {
+        const int64_t n = i / k16, k = (i - n * k16) * 16;
+        off[u] = n * K + k;
+        s[u] = block > 0 ? __ldg(s_inv + (n / block) * nbk + k / block) : __ldg(s_inv);
+        c[u] = ldg_stream(reinterpret_cast<const uint4*>(q + off[u]));
+      }
     }
-    uint4* dst = reinterpret_cast<uint4*>(w + n * K + k);
-    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
-    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (off[u] < 0) continue;
+      const uint32_t cw[4] = {c[u].x, c[u].y, c[u].z, c[u].w};
+      uint32_t o[8];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 a = fp8x2_to_f32<FMT>(uint16_t(cw[j] & 0xFFFFu));
+        const float2 b = fp8x2_to_f32<FMT>(uint16_t(cw[j] >> 16));
+        o[2 * j] = bf16x2_rn(__fmul_rn(a.x, s[u]), __fmul_rn(a.y, s[u]));
+        o[2 * j + 1] = bf16x2_rn(__fmul_rn(b.x, s[u]), __fmul_rn(b.y, s[u]));
+      }
+      uint4* dst = reinterpret_cast<uint4*>(w + off[u]);
+      dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+      dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+    }
   }
 }
 
