@@ -430,13 +430,14 @@ def measure_rows(dev, peaks):
 
     def moe_step():
         F.fp8_moe_route(scores, p["topk"], route["ids"], route["w"], route["offsets"], route["row_token"],
-                        route["row_weight"], route["token_row"])
+                        route["row_weight"], route["token_row"], route["workspace"])
         F.fp8_act_quant_permute(xt, route, qt, st_)
         F.fp8_moe_gemm(qt, st_, qwe, swe, route, out)
 
     ms_f = time_launches(moe_step, 5)
     ms_r = time_launches(lambda: F.fp8_moe_route(scores, p["topk"], route["ids"], route["w"], route["offsets"],
-                                                 route["row_token"], route["row_weight"], route["token_row"]), 10)
+                                                 route["row_token"], route["row_weight"], route["token_row"],
+                                                 route["workspace"]), 10)
     fl_m = 2.0 * p["T"] * p["topk"] * N * K
     res["moe layer (route + act_quant_permute + GEMM with weighted scatter) 4096 tok top-8/256"] = {
         "us": round(ms_f * 1e3, 1), "TFLOPS": round(fl_m / ms_f / 1e9, 1), "route_us": round(ms_r * 1e3, 1)}

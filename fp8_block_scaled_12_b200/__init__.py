@@ -24,6 +24,7 @@ __all__ = [
     "fp8_mx_pack_pow2", "fp8_delayed_quant", "DelayedScaling", "AMAX_MOST_RECENT", "AMAX_MAX",
     "fp8_block_gemm_quant", "fp8_weight_dequant", "block_gemm_quant", "weight_dequant",
     "fp8_moe_route", "fp8_moe_gemm", "fp8_act_quant_permute", "moe_route", "moe_gemm", "act_quant_permute",
+    "moe_route_ws_bytes",
     "fp8_status_string", "fp8_device_error", "fp8_selftest_bounded_wait", "fp8_set_wait_limit_ns",
     "act_quant", "weight_quant", "block_gemm", "grouped_gemm", "mx_quant", "mx_gemm", "mx_pack_pow2",
     "mx_sf_bytes", "EXPORTS",
@@ -65,7 +66,7 @@ def _load() -> ctypes.CDLL:
     L.fp8_delayed_quant.argtypes = [vp, i64, ci, ctypes.c_float, i64, ci, vp, vp, vp, vp, vp, vp, vp]
     L.fp8_block_gemm_quant.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, ci, ci, vp, vp, vp]
     L.fp8_weight_dequant.argtypes = [vp, vp, i64, i64, ci, ci, vp, vp]
-    L.fp8_moe_route.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp, vp, vp]
+    L.fp8_moe_route.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp, vp, vp, i64, vp]
     L.fp8_moe_gemm.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, vp, vp]
     L.fp8_act_quant_permute.argtypes = [vp, i64, i64, i64, ci, ci, vp, i64, vp, vp, vp]
     L.fp8_status_string.argtypes = [ci]
@@ -223,10 +224,17 @@ def fp8_weight_dequant(q: torch.Tensor, s_inv: torch.Tensor, w: torch.Tensor, bl
                                                         _stream(stream)))
 
 
+def moe_route_ws_bytes(T: int, k: int, E: int) -> int:
+    """Workspace of fp8_moe_route (FP8_MOE_ROUTE_WS_BYTES)."""
+    return ((T * k + 511) // 512 + 1) * E * 4
+
+
 def fp8_moe_route(scores: torch.Tensor, k: int, ids: torch.Tensor, w: torch.Tensor, offsets: torch.Tensor,
-                  row_token: torch.Tensor, row_weight: torch.Tensor, token_row: torch.Tensor, stream=None) -> None:
-    """Top-k routing of fp32 scores [T, E], gate weights, and the stable expert sort."""
-    for t in (scores, ids, w, offsets, row_token, row_weight, token_row):
+                  row_token: torch.Tensor, row_weight: torch.Tensor, token_row: torch.Tensor,
+                  workspace: torch.Tensor, stream=None) -> None:
+    """Top-k routing of fp32 scores [T, E], gate weights, and the stable expert sort
+    (workspace: a device buffer of at least moe_route_ws_bytes(T, k, E) bytes)."""
+    for t in (scores, ids, w, offsets, row_token, row_weight, token_row, workspace):
         assert t.is_contiguous()
     T, E = scores.shape
     _expect(scores, (T, E), "scores", torch.float32)
@@ -236,8 +244,10 @@ def fp8_moe_route(scores: torch.Tensor, k: int, ids: torch.Tensor, w: torch.Tens
     for t, n, d in ((row_token, "row_token", torch.int32), (row_weight, "row_weight", torch.float32),
                     (token_row, "token_row", torch.int32)):
         _expect(t, (T * k,), n, d)
+    nbytes = workspace.numel() * workspace.element_size()
     _check("fp8_moe_route", lib.fp8_moe_route(_ptr(scores), T, E, k, _ptr(ids), _ptr(w), _ptr(offsets),
-                                              _ptr(row_token), _ptr(row_weight), _ptr(token_row), _stream(stream)))
+                                              _ptr(row_token), _ptr(row_weight), _ptr(token_row), _ptr(workspace),
+                                              nbytes, _stream(stream)))
 
 
 def fp8_act_quant_permute(x: torch.Tensor, route: dict, q: torch.Tensor, s: torch.Tensor, fmt: int = E4M3,
@@ -471,8 +481,10 @@ def moe_route(scores: torch.Tensor, k: int, stream=None) -> dict:
              offsets=torch.empty((E + 1,), dtype=torch.int32, device=dev),
              row_token=torch.empty((T * k,), dtype=torch.int32, device=dev),
              row_weight=torch.empty((T * k,), dtype=torch.float32, device=dev),
-             token_row=torch.empty((T * k,), dtype=torch.int32, device=dev))
-    fp8_moe_route(scores, k, r["ids"], r["w"], r["offsets"], r["row_token"], r["row_weight"], r["token_row"], stream)
+             token_row=torch.empty((T * k,), dtype=torch.int32, device=dev),
+             workspace=torch.empty((moe_route_ws_bytes(T, k, E) // 4,), dtype=torch.int32, device=dev))
+    fp8_moe_route(scores, k, r["ids"], r["w"], r["offsets"], r["row_token"], r["row_weight"], r["token_row"],
+                  r["workspace"], stream)
     return r
 
 

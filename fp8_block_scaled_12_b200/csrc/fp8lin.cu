@@ -165,6 +165,32 @@ int launch_wide(const void* qa, const void* qw, const GemmArgs& a, cudaStream_t 
   return cuda_status(launch(kern, grid, kThreads, C::SMEM, st, ma, mb, a));
 }
 
+// ------------------------------------------------------ MoE routing
+int launch_moe_route(const float* scores, int64_t T, int64_t E, int64_t k, int32_t* ids, float* w, int32_t* offsets,
+                     int32_t* row_token, float* row_weight, int32_t* token_row, int32_t* ws, cudaStream_t st) {
+  const int64_t P = T * k;
+  const int G = int((P + kMoeChunk - 1) / kMoeChunk);
+  if (T > 0) {
+    const unsigned blocks = unsigned((T * 32 + 255) / 256);
+    const cudaError_t e = E <= 256 ? launch(k_moe_topk<8>, blocks, 256, 0, st, scores, int(T), int(E), int(k), ids, w)
+                                   : launch(k_moe_topk<32>, blocks, 256, 0, st, scores, int(T), int(E), int(k), ids, w);
+    if (e != cudaSuccess) return FP8_ERR_CUDA;
+  }
+  const size_t smem = size_t(1 + kMoeSortThreads / 32) * size_t(E) * sizeof(int32_t);
+  if (G <= 1)   // every pair in one chunk: one CTA sorts them all
+    return cuda_status(launch(k_moe_place<true>, 1, kMoeSortThreads, smem, st, static_cast<const int32_t*>(ids),
+                              static_cast<const float*>(w), P, int(k), int(E), G, static_cast<const int32_t*>(ws),
+                              offsets, row_token, row_weight, token_row));
+  if (launch(k_moe_count, unsigned(G), kMoeSortThreads, size_t(E) * 4, st, static_cast<const int32_t*>(ids), P,
+             int(E), ws) != cudaSuccess)
+    return FP8_ERR_CUDA;
+  const unsigned sblocks = unsigned((E + kMoeSortThreads / 32 - 1) / (kMoeSortThreads / 32));
+  if (launch(k_moe_scan, sblocks, kMoeSortThreads, 0, st, G, int(E), ws) != cudaSuccess) return FP8_ERR_CUDA;
+  return cuda_status(launch(k_moe_place<false>, unsigned(G), kMoeSortThreads, smem, st,
+                            static_cast<const int32_t*>(ids), static_cast<const float*>(w), P, int(k), int(E), G,
+                            static_cast<const int32_t*>(ws), offsets, row_token, row_weight, token_row));
+}
+
 // ------------------------------------------------------ quantiser launches
 template <int FMT, int SF>
 int launch_act_quant(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q, float* s,
@@ -479,26 +505,18 @@ int fp8_mx_pack_pow2(const float* s, int64_t rows, int64_t K, int row_block, voi
 }
 
 int fp8_moe_route(const float* scores, int64_t T, int64_t E, int64_t k, int32_t* ids, float* w, int32_t* offsets,
-                  int32_t* row_token, float* row_weight, int32_t* token_row, void* stream) {
+                  int32_t* row_token, float* row_weight, int32_t* token_row, void* workspace, int64_t workspace_bytes,
+                  void* stream) {
   if (T < 0 || E < 1 || E > kMoeMaxE || k < 1 || k > kMoeMaxK || k > E) return FP8_ERR_INVALID_ARG;
   if (T * k > INT32_MAX) return FP8_ERR_SHAPE;
-  if (!offsets) return FP8_ERR_INVALID_ARG;
+  if (!offsets || !workspace) return FP8_ERR_INVALID_ARG;
   if (T > 0 && (!scores || !ids || !w || !row_token || !row_weight || !token_row)) return FP8_ERR_INVALID_ARG;
   if (!aligned(scores, 4) || !aligned(ids, 4) || !aligned(w, 4) || !aligned(offsets, 4) || !aligned(row_token, 4) ||
-      !aligned(row_weight, 4) || !aligned(token_row, 4))
+      !aligned(row_weight, 4) || !aligned(token_row, 4) || !aligned(workspace, 4))
     return FP8_ERR_ALIGNMENT;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (T > 0) {
-    const int blocks = int((T * 32 + 255) / 256);
-    const cudaError_t e = E <= 256 ? launch(k_moe_topk<8>, unsigned(blocks), 256, 0, st, scores, int(T), int(E), int(k), ids, w)
-                                   : launch(k_moe_topk<32>, unsigned(blocks), 256, 0, st, scores, int(T), int(E), int(k), ids, w);
-    if (e != cudaSuccess) return FP8_ERR_CUDA;
-  }
-  const size_t smem = size_t(32) * size_t(E) * sizeof(int32_t);
-  if (cudaFuncSetAttribute(k_moe_sort, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
-    return FP8_ERR_CUDA;
-  return cuda_status(launch(k_moe_sort, 1, 1024, smem, st, static_cast<const int32_t*>(ids), static_cast<const float*>(w),
-                            int(T), int(E), int(k), offsets, row_token, row_weight, token_row));
+  if (workspace_bytes < FP8_MOE_ROUTE_WS_BYTES(T, k, E)) return FP8_ERR_SHAPE;
+  return launch_moe_route(scores, T, E, k, ids, w, offsets, row_token, row_weight, token_row,
+                          static_cast<int32_t*>(workspace), static_cast<cudaStream_t>(stream));
 }
 
 int fp8_act_quant_permute(const void* x, int64_t T, int64_t K, int64_t ldx, int fmt, int scale_fmt,

@@ -274,10 +274,18 @@ int fp8_delayed_quant(const void* x, int64_t n, int fmt, float target, int64_t h
  *   offsets    int32 [E+1]: rows of expert e are [offsets[e], offsets[e+1]).
  *   row_token, row_weight   int32 / fp32 [T*k]: token and gate weight of each sorted row.
  *   token_row  int32 [T*k]: sorted row of pair (t, j) at t*k + j.
- * No global scratch: one kernel per token group picks the experts, one CTA sorts.
+ *   workspace  DEVICE scratch owned by the caller, at least FP8_MOE_ROUTE_WS_BYTES(T, k, E)
+ *              bytes, 4-byte aligned, no initial contents required; it carries the
+ *              per-chunk expert counts of the sort (chunks of 512 pairs, one CTA each),
+ *              so calls that share a workspace must be ordered on one stream.
+ * Returns FP8_OK or an error status (FP8_ERR_SHAPE for a workspace that is too small).
  */
+#define FP8_MOE_ROUTE_WS_BYTES(T, k, E) \
+  (((((int64_t)(T) * (int64_t)(k)) + 511) / 512 + 1) * (int64_t)(E) * 4)
+
 int fp8_moe_route(const float* scores, int64_t T, int64_t E, int64_t k, int32_t* ids, float* w, int32_t* offsets,
-                  int32_t* row_token, float* row_weight, int32_t* token_row, void* stream);
+                  int32_t* row_token, float* row_weight, int32_t* token_row, void* workspace, int64_t workspace_bytes,
+                  void* stream);
 
 /*
  * fp8_act_quant_permute -- fp8_act_quant (group 128) of the T token rows of x, each

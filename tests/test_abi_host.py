@@ -212,12 +212,18 @@ def test_fused_and_dequant_validation():
 
 def test_moe_validation():
     mr = F.lib.fp8_moe_route
-    # (scores, T, E, k, ids, w, offsets, row_token, row_weight, token_row, stream)
-    assert mr(FAKE, 16, 0, 2, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, S) == INVALID       # E
-    assert mr(FAKE, 16, 2048, 8, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, S) == INVALID    # E > 1024
-    assert mr(FAKE, 16, 8, 9, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, S) == INVALID       # k > E
-    assert mr(FAKE, 16, 8, 33, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, S) == INVALID      # k > 32
-    assert mr(FAKE + 2, 16, 8, 2, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, S) == ALIGN
+    # (scores, T, E, k, ids, w, offsets, row_token, row_weight, token_row, workspace, ws_bytes, stream)
+    ws = F.moe_route_ws_bytes(16, 8, 1024)
+    assert mr(FAKE, 16, 0, 2, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ws, S) == INVALID       # E
+    assert mr(FAKE, 16, 2048, 8, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ws, S) == INVALID    # E > 1024
+    assert mr(FAKE, 16, 8, 9, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ws, S) == INVALID       # k > E
+    assert mr(FAKE, 16, 8, 33, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ws, S) == INVALID      # k > 32
+    assert mr(FAKE, 16, 8, 2, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, ws, S) == INVALID       # no workspace
+    assert mr(FAKE + 2, 16, 8, 2, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ws, S) == ALIGN
+    assert mr(FAKE, 16, 8, 2, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 2, ws, S) == ALIGN
+    # workspace: (ceil(T*k / 512) + 1) * E int32
+    assert F.moe_route_ws_bytes(4096, 8, 256) == (64 + 1) * 256 * 4
+    assert mr(FAKE, 4096, 256, 8, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 65 * 256 * 4 - 4, S) == SHAPE
     mg = F.lib.fp8_moe_gemm
     # (qa, sa, qw, sw, offsets, row_token, row_weight, T, E, k, N, K, out, stream)
     assert mg(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 16, 4, 2, 256, 200, FAKE, S) == SHAPE   # K % 128

@@ -51,6 +51,19 @@ def test_routing_ties(cuda_device):
     route_both(cuda_device, scores_for(1000, 256, seed=1, ties=True), 8)
 
 
+def test_routing_many_chunks(cuda_device):
+    """131072 pairs: 256 chunks of the sort, each placing its rows after all earlier
+    chunks' rows of the same expert."""
+    route_both(cuda_device, scores_for(16384, 256, seed=5), 8)
+
+
+def test_routing_no_tokens(cuda_device):
+    r = F.moe_route(torch.empty((0, 64), dtype=torch.float32, device=cuda_device), 4)
+    torch.cuda.synchronize()
+    assert F.fp8_device_error() == 0
+    assert r["offsets"].cpu().tolist() == [0] * 65
+
+
 def moe_compare(dev, T, E, k, N, K, seed, tokens=None):
     scores = scores_for(T, E, seed)
     r, ro = route_both(dev, scores, k)
