@@ -24,7 +24,7 @@ __all__ = [
     "fp8_mx_pack_pow2", "fp8_delayed_quant", "DelayedScaling", "AMAX_MOST_RECENT", "AMAX_MAX",
     "fp8_block_gemm_quant", "fp8_weight_dequant", "block_gemm_quant", "weight_dequant",
     "fp8_moe_route", "fp8_moe_gemm", "fp8_act_quant_permute", "moe_route", "moe_gemm", "act_quant_permute",
-    "moe_route_ws_bytes",
+    "moe_route_ws_bytes", "fp8_moe_route_noalloc", "moe_route_noalloc",
     "fp8_status_string", "fp8_device_error", "fp8_selftest_bounded_wait", "fp8_set_wait_limit_ns",
     "act_quant", "weight_quant", "block_gemm", "grouped_gemm", "mx_quant", "mx_gemm", "mx_pack_pow2",
     "mx_sf_bytes", "EXPORTS",
@@ -67,6 +67,7 @@ def _load() -> ctypes.CDLL:
     L.fp8_block_gemm_quant.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, ci, ci, vp, vp, vp]
     L.fp8_weight_dequant.argtypes = [vp, vp, i64, i64, ci, ci, vp, vp]
     L.fp8_moe_route.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp, vp, vp, i64, vp]
+    L.fp8_moe_route_noalloc.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp, vp, vp]
     L.fp8_moe_gemm.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, vp, vp]
     L.fp8_act_quant_permute.argtypes = [vp, i64, i64, i64, ci, ci, vp, i64, vp, vp, vp]
     L.fp8_status_string.argtypes = [ci]
@@ -248,6 +249,25 @@ def fp8_moe_route(scores: torch.Tensor, k: int, ids: torch.Tensor, w: torch.Tens
     _check("fp8_moe_route", lib.fp8_moe_route(_ptr(scores), T, E, k, _ptr(ids), _ptr(w), _ptr(offsets),
                                               _ptr(row_token), _ptr(row_weight), _ptr(token_row), _ptr(workspace),
                                               nbytes, _stream(stream)))
+
+
+def fp8_moe_route_noalloc(scores: torch.Tensor, k: int, ids: torch.Tensor, w: torch.Tensor, offsets: torch.Tensor,
+                          row_token: torch.Tensor, row_weight: torch.Tensor, token_row: torch.Tensor,
+                          stream=None) -> None:
+    """fp8_moe_route with the library's own fixed scratch (no workspace argument)."""
+    for t in (scores, ids, w, offsets, row_token, row_weight, token_row):
+        assert t.is_contiguous()
+    T, E = scores.shape
+    _expect(scores, (T, E), "scores", torch.float32)
+    _expect(ids, (T, k), "ids", torch.int32)
+    _expect(w, (T, k), "w", torch.float32)
+    _expect(offsets, (E + 1,), "offsets", torch.int32)
+    for t, n, d in ((row_token, "row_token", torch.int32), (row_weight, "row_weight", torch.float32),
+                    (token_row, "token_row", torch.int32)):
+        _expect(t, (T * k,), n, d)
+    _check("fp8_moe_route_noalloc", lib.fp8_moe_route_noalloc(_ptr(scores), T, E, k, _ptr(ids), _ptr(w),
+                                                              _ptr(offsets), _ptr(row_token), _ptr(row_weight),
+                                                              _ptr(token_row), _stream(stream)))
 
 
 def fp8_act_quant_permute(x: torch.Tensor, route: dict, q: torch.Tensor, s: torch.Tensor, fmt: int = E4M3,
@@ -485,6 +505,20 @@ def moe_route(scores: torch.Tensor, k: int, stream=None) -> dict:
              workspace=torch.empty((moe_route_ws_bytes(T, k, E) // 4,), dtype=torch.int32, device=dev))
     fp8_moe_route(scores, k, r["ids"], r["w"], r["offsets"], r["row_token"], r["row_weight"], r["token_row"],
                   r["workspace"], stream)
+    return r
+
+
+def moe_route_noalloc(scores: torch.Tensor, k: int, stream=None) -> dict:
+    T, E = scores.shape
+    dev = scores.device
+    r = dict(ids=torch.empty((T, k), dtype=torch.int32, device=dev),
+             w=torch.empty((T, k), dtype=torch.float32, device=dev),
+             offsets=torch.empty((E + 1,), dtype=torch.int32, device=dev),
+             row_token=torch.empty((T * k,), dtype=torch.int32, device=dev),
+             row_weight=torch.empty((T * k,), dtype=torch.float32, device=dev),
+             token_row=torch.empty((T * k,), dtype=torch.int32, device=dev))
+    fp8_moe_route_noalloc(scores, k, r["ids"], r["w"], r["offsets"], r["row_token"], r["row_weight"], r["token_row"],
+                          stream)
     return r
 
 

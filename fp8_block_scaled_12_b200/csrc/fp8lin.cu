@@ -519,6 +519,46 @@ int fp8_moe_route(const float* scores, int64_t T, int64_t E, int64_t k, int32_t*
                           static_cast<int32_t*>(workspace), static_cast<cudaStream_t>(stream));
 }
 
+// ------------------------------------------------------ routing without a caller workspace
+// The sort's scratch in a file-scope device array of fixed size: 256 KiB, i.e. (G + 1) * E
+// <= 65536 int32 for G = ceil(T*k / 512) chunks (e.g. 4096 tokens, top-8 of 256 experts:
+// 65 x 256).  One array per device, shared by every call on that device.
+constexpr int64_t kRouteScratchInts = 65536;
+constexpr int kRouteMaxDevices = 64;
+static __device__ __align__(256) int32_t g_route_scratch[kRouteScratchInts];
+
+int fp8_moe_route_noalloc(const float* scores, int64_t T, int64_t E, int64_t k, int32_t* ids, float* w,
+                          int32_t* offsets, int32_t* row_token, float* row_weight, int32_t* token_row, void* stream) {
+  if (T < 0 || E < 1 || E > kMoeMaxE || k < 1 || k > kMoeMaxK || k > E) return FP8_ERR_INVALID_ARG;
+  if (T * k > INT32_MAX) return FP8_ERR_SHAPE;
+  if (FP8_MOE_ROUTE_WS_BYTES(T, k, E) > kRouteScratchInts * int64_t(sizeof(int32_t))) return FP8_ERR_SHAPE;
+  if (!offsets) return FP8_ERR_INVALID_ARG;
+  if (T > 0 && (!scores || !ids || !w || !row_token || !row_weight || !token_row)) return FP8_ERR_INVALID_ARG;
+  if (!aligned(scores, 4) || !aligned(ids, 4) || !aligned(w, 4) || !aligned(offsets, 4) || !aligned(row_token, 4) ||
+      !aligned(row_weight, 4) || !aligned(token_row, 4))
+    return FP8_ERR_ALIGNMENT;
+  // the array's device address, looked up once per device with that device current
+  static std::mutex mu;
+  static int32_t* scratch[kRouteMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kRouteMaxDevices) return FP8_ERR_CUDA;
+  int32_t* ws;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!scratch[dev]) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || !p) return FP8_ERR_CUDA;
+      scratch[dev] = static_cast<int32_t*>(p);
+    }
+    ws = scratch[dev];
+  }
+  // every workspace entry the passes read is written earlier in the same call (the count
+  // pass writes each chunk's full histogram row, the scan pass the totals row), so
+  // nothing has to start at zero and nothing is cleared
+  return launch_moe_route(scores, T, E, k, ids, w, offsets, row_token, row_weight, token_row, ws,
+                          static_cast<cudaStream_t>(stream));
+}
+
 int fp8_act_quant_permute(const void* x, int64_t T, int64_t K, int64_t ldx, int fmt, int scale_fmt,
                           const int32_t* token_row, int64_t k, void* q, float* s, void* stream) {
   if (T < 0 || K <= 0 || ldx < K || k < 1 || k > kMoeMaxK) return FP8_ERR_INVALID_ARG;

@@ -288,6 +288,21 @@ int fp8_moe_route(const float* scores, int64_t T, int64_t E, int64_t k, int32_t*
                   void* stream);
 
 /*
+ * fp8_moe_route_noalloc -- fp8_moe_route with the sort's scratch inside the library
+ * instead of a caller workspace; the pages have no counterpart (it is an interface
+ * variant, not a step of the method).  Same arguments and results as fp8_moe_route,
+ * without workspace / workspace_bytes.  The scratch is a fixed device array of 256 KiB
+ * per device: problems with FP8_MOE_ROUTE_WS_BYTES(T, k, E) > 262144 are rejected with
+ * FP8_ERR_SHAPE (e.g. 4096 tokens, top-8 of 256 experts fit; 16384 tokens do not).  The
+ * array's address is looked up once per device (with that device current); the call
+ * allocates and frees no memory, and nothing in the array has to start at zero.  All
+ * calls on one device share the array, so calls that overlap in time (different
+ * streams, or host threads without ordering) race and give undefined results.
+ */
+int fp8_moe_route_noalloc(const float* scores, int64_t T, int64_t E, int64_t k, int32_t* ids, float* w,
+                          int32_t* offsets, int32_t* row_token, float* row_weight, int32_t* token_row, void* stream);
+
+/*
  * fp8_act_quant_permute -- fp8_act_quant (group 128) of the T token rows of x, each
  * row's codes and scales written to its k expert-sorted rows token_row[t*k + j]
  * (fp8_moe_route's map).  Per-token quantisation commutes with duplicating a row, so

@@ -224,6 +224,12 @@ def test_moe_validation():
     # workspace: (ceil(T*k / 512) + 1) * E int32
     assert F.moe_route_ws_bytes(4096, 8, 256) == (64 + 1) * 256 * 4
     assert mr(FAKE, 4096, 256, 8, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 65 * 256 * 4 - 4, S) == SHAPE
+    mn = F.lib.fp8_moe_route_noalloc
+    # (scores, T, E, k, ids, w, offsets, row_token, row_weight, token_row, stream): the
+    # library's scratch holds 65536 int32; (256 + 1) * 256 of them do not fit
+    assert mn(FAKE, 16384, 256, 8, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, S) == SHAPE
+    assert mn(FAKE, 16, 8, 9, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, S) == INVALID
+    assert mn(FAKE + 2, 16, 8, 2, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, S) == ALIGN
     mg = F.lib.fp8_moe_gemm
     # (qa, sa, qw, sw, offsets, row_token, row_weight, T, E, k, N, K, out, stream)
     assert mg(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 16, 4, 2, 256, 200, FAKE, S) == SHAPE   # K % 128
