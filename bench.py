@@ -562,6 +562,27 @@ def measure_mx_rows(dev, peaks):
         b = 18432 * 7168 + ewd.numel() + Md * (7168 + 56 * 4 + 18432 * 2)
         res[f"mx_gemm ue8m0 decode M={Md} (pack + gemm)"] = {"us": round(ms * 1e3, 2), "GB/s": round(b / ms / 1e6, 1),
                                                             "frac_hbm": round(b / ms / 1e6 / hbm, 4)}
+    del wds
+    # decode on MXFP8 operands (E8M0 per 32 elements on both sides), two weight copies
+    wms = []
+    for c in range(2):
+        wd = synth.weights(18432, 7168, 0.015, seed=c, device=dev)
+        wms.append(F.mx_quant(wd))
+        del wd
+    for Md in (1, 64):
+        xd = synth.activations(Md, 7168, seed=0, device=dev)
+        qa, ea = F.mx_quant(xd)
+        y = torch.empty((Md, 18432), dtype=torch.bfloat16, device=dev)
+        turn = itertools.cycle(wms)
+
+        def mstep():
+            qwm, ewm = next(turn)
+            F.fp8_mx_gemm(qa, ea, qwm, ewm, y)
+
+        ms = time_launches(mstep, 20)
+        b = 18432 * 7168 + wms[0][1].numel() + Md * (7168 + 7168 // 32 + 18432 * 2)
+        res[f"mx_gemm e8m0x32 decode M={Md}"] = {"us": round(ms * 1e3, 2), "GB/s": round(b / ms / 1e6, 1),
+                                               "frac_hbm": round(b / ms / 1e6 / hbm, 4)}
     assert F.fp8_device_error() == 0
     return res
 
