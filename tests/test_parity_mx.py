@@ -132,6 +132,13 @@ def test_mx_gemm_token_counts(cuda_device, M):
     mx_gemm_compare(cuda_device, M, 384, 1024, seed=M)
 
 
+@pytest.mark.parametrize("M", [1, 40, 100, 300])
+def test_mx_gemm_single_k_block(cuda_device, M):
+    """K = 128: the weight-stationary shapes' second MMA issuer gets no K-block, so the
+    epilogue must use the first accumulator alone."""
+    mx_gemm_compare(cuda_device, M, 384, 128, seed=M + 7)
+
+
 @pytest.mark.parametrize("shape", [(257, 512, 512), (300, 272, 640), (1000, 528, 384), (40, 272, 7296)])
 def test_mx_gemm_ragged(cuda_device, shape):
     M, N, K = shape
