@@ -64,8 +64,8 @@ def test_routing_no_tokens(cuda_device):
     assert r["offsets"].cpu().tolist() == [0] * 65
 
 
-def moe_compare(dev, T, E, k, N, K, seed, tokens=None):
-    scores = scores_for(T, E, seed)
+def moe_compare(dev, T, E, k, N, K, seed, tokens=None, scores=None):
+    scores = scores_for(T, E, seed) if scores is None else scores
     r, ro = route_both(dev, scores, k)
     x = synth.activations(T, K, seed=seed, device=dev)
     qa, sa = F.act_quant(x)                      # token-major, for the oracle's combine
@@ -102,3 +102,18 @@ def test_moe_config_full_size(cuda_device):
     p = synth.MOE.params
     toks = np.linspace(0, p["T"] - 1, 48).astype(np.int64)
     moe_compare(cuda_device, p["T"], p["E"], p["topk"], p["N"], p["K"], seed=0, tokens=toks)
+
+
+def test_moe_skewed_experts(cuda_device):
+    """Expert 0 preferred by most tokens: its 560+ rows span four chunks of 160 in the
+    scatter GEMM, while other experts get a few rows or none."""
+    T, E, k = 700, 16, 2
+    s = scores_for(T, E, seed=13)
+    s[:600, 0] += 2.0                                   # expert 0 wins for 600 tokens
+    moe_compare(cuda_device, T, E, k, 256, 512, seed=13, scores=s)
+
+
+@pytest.mark.parametrize("T,E,k", [(200, 8, 1), (50, 4, 4)])
+def test_moe_top1_and_all_experts(cuda_device, T, E, k):
+    """k = 1 (each token one expert, weight 1) and k = E (every expert every token)."""
+    moe_compare(cuda_device, T, E, k, 256, 512, seed=T + k)
