@@ -343,6 +343,35 @@ def time_launches(fn, iters, warm=2):
     return a.elapsed_time(b) / iters
 
 
+def time_graph(fn, iters, warm=2):
+    """Device time per call of `fn` with `iters` calls captured in one CUDA graph and
+    replayed: what a serving loop that launches through graphs sees, free of the
+    Python / ctypes launch overhead that bounds microsecond-scale kernels eagerly."""
+    import torch
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        fn()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(iters):
+            fn()
+    g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    del g
+    return a.elapsed_time(b) / iters
+
+
 def measure_rows(dev, peaks):
     """Every hot-path row on its own configuration (CUDA events, a few launches each)."""
     import torch
@@ -382,10 +411,12 @@ def measure_rows(dev, peaks):
                 xi, qi, si, _ = next(turn)
                 F.fp8_act_quant(xi, qi, si, scale_fmt=sf)
 
-            ms = time_launches(aq, 4 * nsets)
+            ms_e = time_launches(aq, 4 * nsets)
+            ms = time_graph(aq, 4 * nsets)
             b = Ms * K * 3 + Ms * (K // 128) * 4
             res[f"{name} {Ms}x7168"] = {"GB/s": round(b / ms / 1e6, 1), "frac_hbm": round(b / ms / 1e6 / hbm, 4),
-                                        "us": round(ms * 1e3, 2)}
+                                        "us": round(ms * 1e3, 2), "timing": "CUDA graph replay",
+                                        "us_eager": round(ms_e * 1e3, 2)}
         for name, fmt in (("per_tensor_e4m3", F.E4M3), ("per_tensor_e5m2", F.E5M2)):
             turn = itertools.cycle(sets)
 
@@ -393,10 +424,12 @@ def measure_rows(dev, peaks):
                 xi, qi, _, s1i = next(turn)
                 F.fp8_weight_quant(xi, qi, s1i, block=0, fmt=fmt)
 
-            ms = time_launches(pt, 4 * nsets)
+            ms_e = time_launches(pt, 4 * nsets)
+            ms = time_graph(pt, 4 * nsets)
             b = Ms * K * 3 + 4
             res[f"{name} {Ms}x7168"] = {"GB/s (algorithmic 3 B/elt)": round(b / ms / 1e6, 1),
-                                        "frac_hbm": round(b / ms / 1e6 / hbm, 4), "us": round(ms * 1e3, 2)}
+                                        "frac_hbm": round(b / ms / 1e6 / hbm, 4), "us": round(ms * 1e3, 2),
+                                        "timing": "CUDA graph replay", "us_eager": round(ms_e * 1e3, 2)}
         del sets
     # delayed scaling: one pass, previous step's scale, amax history of 16 (3 B/elt + state)
     ds = F.DelayedScaling(hist_len=16, device=dev)
@@ -435,10 +468,12 @@ def measure_rows(dev, peaks):
             F.fp8_block_gemm(qa, sa, qwd, swd_, y)
 
         ms = time_launches(dgemm, 20)
+        ms_g = time_graph(dgemm, 20)
         b = 18432 * 7168 + swd.numel() * 4 + Md * (7168 + 56 * 4 + 18432 * 2)
         res[f"decode_gemm M={Md}"] = {"us": round(ms * 1e3, 2), "GB/s": round(b / ms / 1e6, 1),
                                       "frac_hbm": round(b / ms / 1e6 / hbm, 4),
-                                      "TFLOPS": round(2 * Md * 18432 * 7168 / ms / 1e9, 2)}
+                                      "TFLOPS": round(2 * Md * 18432 * 7168 / ms / 1e9, 2),
+                                      "us_graph": round(ms_g * 1e3, 2), "frac_hbm_graph": round(b / ms_g / 1e6 / hbm, 4)}
     del wds, swd
     # grouped MoE GEMM
     p = synth.MOE.params
@@ -612,9 +647,12 @@ def measure_mx_rows(dev, peaks):
             F.fp8_mx_gemm(qa, ea, qwm, ewm, y)
 
         ms = time_launches(mstep, 20)
+        ms_g = time_graph(mstep, 20)
         b = 18432 * 7168 + wms[0][1].numel() + Md * (7168 + 7168 // 32 + 18432 * 2)
         res[f"mx_gemm e8m0x32 decode M={Md}"] = {"us": round(ms * 1e3, 2), "GB/s": round(b / ms / 1e6, 1),
-                                               "frac_hbm": round(b / ms / 1e6 / hbm, 4)}
+                                               "frac_hbm": round(b / ms / 1e6 / hbm, 4),
+                                               "us_graph": round(ms_g * 1e3, 2),
+                                               "frac_hbm_graph": round(b / ms_g / 1e6 / hbm, 4)}
     assert F.fp8_device_error() == 0
     return res
 
