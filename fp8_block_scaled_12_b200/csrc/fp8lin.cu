@@ -5,6 +5,7 @@
 
 #include <cstdint>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "../../include/fp8lin.h"
@@ -108,6 +109,23 @@ bool launch_regs_ok(K kern) {
   return fa.numRegs == int(kLaunchRegs);
 }
 
+// The register check and the dynamic shared-memory limit of a warp-specialised kernel
+// persist in the device's context, so they run on its first launch per device only
+// (`ready`: one bit per device, owned by the calling launch function; devices past 63
+// are set up on every launch).
+template <typename K>
+int kernel_setup(std::atomic<uint64_t>& ready, K kern, size_t smem) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FP8_ERR_CUDA;
+  const uint64_t bit = (dev >= 0 && dev < 64) ? (uint64_t(1) << dev) : 0u;
+  if (bit != 0u && (ready.load(std::memory_order_acquire) & bit) != 0u) return FP8_OK;
+  if (!launch_regs_ok(kern)) return FP8_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
+    return FP8_ERR_CUDA;
+  ready.fetch_or(bit, std::memory_order_acq_rel);
+  return FP8_OK;
+}
+
 template <int NT, int NBUF, int STAGES, int KB_CAP, bool QOUT = false, bool MOE = false>
 int launch_swap(const void* qa, const void* qw, const GemmArgs& a, int64_t w_rows, cudaStream_t st) {
   using C = SwapCfg<NT, NBUF, STAGES, KB_CAP>;
@@ -117,9 +135,8 @@ int launch_swap(const void* qa, const void* qw, const GemmArgs& a, int64_t w_row
   if (!make_map_u8(&mw, qw, uint64_t(w_rows), uint64_t(a.K), 128)) return FP8_ERR_CUDA;
   if (!make_map_u8(&mx, qa, uint64_t(a.M > 0 ? a.M : 1), uint64_t(a.K), 32)) return FP8_ERR_CUDA;
   auto kern = k_gemm_swap<NT, NBUF, STAGES, KB_CAP, QOUT, MOE>;
-  if (!launch_regs_ok(kern)) return FP8_ERR_UNSUPPORTED;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-  if (e != cudaSuccess) return FP8_ERR_CUDA;
+  static std::atomic<uint64_t> ready{0};
+  if (const int st_ = kernel_setup(ready, kern, smem)) return st_;
   const int nbn = (a.N + 127) / 128;
   const int64_t units = int64_t(a.E) * nbn;
   const int grid = int(units < num_sms() ? units : num_sms());
@@ -141,9 +158,8 @@ int launch_mx(const void* qa, const void* qw, const MxArgs& a, cudaStream_t st) 
   if (!make_map_u8(&mp, pp, prow, uint64_t(a.K), 128)) return FP8_ERR_CUDA;
   if (!make_map_u8(&mq, qp, qrow, uint64_t(a.K), SWAP ? 32u : uint32_t(NQ))) return FP8_ERR_CUDA;
   auto kern = k_gemm_mx<C>;
-  if (!launch_regs_ok(kern)) return FP8_ERR_UNSUPPORTED;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-  if (e != cudaSuccess) return FP8_ERR_CUDA;
+  static std::atomic<uint64_t> ready{0};
+  if (const int st_ = kernel_setup(ready, kern, smem)) return st_;
   const int64_t tiles = SWAP ? int64_t((a.N + 127) / 128) * ((a.M + NQ - 1) / NQ)
                              : int64_t((a.M + 127) / 128) * ((a.N + NQ - 1) / NQ);
   const int grid = int(tiles < num_sms() ? tiles : num_sms());
@@ -157,9 +173,8 @@ int launch_wide(const void* qa, const void* qw, const GemmArgs& a, cudaStream_t 
   if (!make_map_u8(&ma, qa, uint64_t(a.M), uint64_t(a.K), C::BM)) return FP8_ERR_CUDA;
   if (!make_map_u8(&mb, qw, uint64_t(a.N), uint64_t(a.K), C::BN)) return FP8_ERR_CUDA;
   auto kern = k_gemm_wide<kWideStages, QOUT>;
-  if (!launch_regs_ok(kern)) return FP8_ERR_UNSUPPORTED;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(C::SMEM));
-  if (e != cudaSuccess) return FP8_ERR_CUDA;
+  static std::atomic<uint64_t> ready{0};
+  if (const int st_ = kernel_setup(ready, kern, size_t(C::SMEM))) return st_;
   const int64_t tiles = int64_t((a.M + C::BM - 1) / C::BM) * ((a.N + C::BN - 1) / C::BN);
   const int grid = int(tiles < num_sms() ? tiles : num_sms());
   return cuda_status(launch(kern, grid, kThreads, C::SMEM, st, ma, mb, a));
