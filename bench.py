@@ -176,6 +176,15 @@ def setup_prefill(dev, rank):
     return dict(M=M, N=N, K=K, x=x, qa=qa, sa=sa, qw=qw, sw=sw, y=y, F=F, desc=synth.PREFILL.desc)
 
 
+def prefill_config(M, N, K, world):
+    """The `config` of the headline line; the reference arm reports the same one (its
+    bounded per-step sample is described in its cpu_baseline.sample)."""
+    return {"workload": f"prefill-shaped linear: act_quant + block-scaled FP8 GEMM, M={M} N={N} K={K}, "
+                        "128-ch act groups, 128x128 weight blocks, fp32 scales, bf16 out",
+            "M_per_gpu": M, "N": N, "K": K, "parallelism": f"dp{world} (token batches)",
+            "l2": "inputs larger than L2 (W 235 MB); no flush"}
+
+
 def run_ours(args, world, rank, local):
     import torch
     import torch.distributed as dist
@@ -246,10 +255,7 @@ def run_ours(args, world, rank, local):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3",
         "data": "synthetic (seeded N(0,1) activations with 1% outlier channels x20, N(0,0.02) weights)",
-        "config": {"workload": "prefill-shaped linear: act_quant + block-scaled FP8 GEMM, "
-                               "M=4096 N=28672 K=8192, 128-ch act groups, 128x128 weight blocks, fp32 scales, "
-                               "bf16 out", "M_per_gpu": M, "N": N, "K": K, "parallelism": f"dp{world} (token batches)",
-                   "l2": "inputs larger than L2 (W 235 MB); no flush"},
+        "config": prefill_config(M, N, K, world),
         "gpu_launches": 2 * args.steps,
         "e2e": {"value": round(e2e_tflops, 2), "unit": "TFLOPS", "h2d_bytes_per_step": M * K * 2,
                 "d2h_bytes_per_step": M * N * 2},
@@ -763,9 +769,7 @@ def run_reference(args, world, rank):
     out = {"impl": "reference", "metric": METRIC, "value": round(v, 6), "unit": "TFLOPS", "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3 / args.steps, 2),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-           "data": "synthetic", "config": {"workload": f"prefill-shaped linear M={M} N={N} K={K} (bounded "
-                                                       f"sample per step: act_quant of 1 row + its GEMM "
-                                                       f"against all {N} weight rows)"},
+           "data": "synthetic", "config": prefill_config(M, N, K, world),
            "cpu_baseline": {"value": round(v, 6), "unit": "TFLOPS", "cores": usable, "host_cores": reported,
                             "kind": "oracle",
                             "sample": f"act_quant of 1 row + fp64 GEMM of 1 row x {N} x {K} per step, "
