@@ -245,3 +245,21 @@ def test_moe_validation():
     assert ap(FAKE, 16, 256, 256, 0, 0, None, 2, FAKE, FAKE, S) == INVALID
     assert ap(FAKE, 16, 256, 256, 0, 0, FAKE + 2, 2, FAKE, FAKE, S) == ALIGN
     assert ap(FAKE, 0, 256, 256, 0, 0, None, 2, None, None, S) == OK
+
+
+def test_header_is_plain_c_and_links(tmp_path):
+    """A C99 program built against include/fp8lin.h and the library (no GPU needed)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    libdir = os.path.dirname(F.LIB_PATH)
+    exe = str(tmp_path / "c_abi_check")
+    cmd = [gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.join(root, "include"),
+           "-o", exe, os.path.join(root, "tests", "c_abi_check.c"), "-L", libdir, "-lfp8lin",
+           "-Wl,-rpath," + libdir]
+    subprocess.run(cmd, check=True, capture_output=True)
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0 and "c abi ok" in r.stdout, (r.returncode, r.stdout, r.stderr)
