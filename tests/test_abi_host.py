@@ -263,3 +263,18 @@ def test_header_is_plain_c_and_links(tmp_path):
     subprocess.run(cmd, check=True, capture_output=True)
     r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
     assert r.returncode == 0 and "c abi ok" in r.stdout, (r.returncode, r.stdout, r.stderr)
+
+
+def test_binding_fails_loudly_without_the_library(tmp_path):
+    """A copy of the binding next to no libfp8lin.so refuses to import (no fallback)."""
+    import shutil
+    import subprocess
+    import sys
+    pkg = tmp_path / "fp8_block_scaled_12_b200"
+    pkg.mkdir()
+    shutil.copy(os.path.join(ROOT, "fp8_block_scaled_12_b200", "__init__.py"), pkg / "__init__.py")
+    r = subprocess.run([sys.executable, "-c", "import fp8_block_scaled_12_b200"], cwd=tmp_path,
+                       capture_output=True, text=True, timeout=300,
+                       env={**os.environ, "PYTHONPATH": str(tmp_path)})
+    assert r.returncode != 0
+    assert "ImportError" in r.stderr and "libfp8lin.so is missing" in r.stderr
