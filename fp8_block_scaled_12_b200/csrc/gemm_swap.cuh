@@ -60,6 +60,13 @@ struct SwapCfg {
 
 constexpr int kSwapIssuersMax = 3;
 
+// Register split of this kernel (same 384 x kLaunchRegs pool as gemm.cuh): its
+// producer and issuer threads walk the segment sequence and need more than 48
+// registers, its epilogue holds at most 96 token columns per thread.
+constexpr uint32_t kSwapProducerRegs = 64;
+constexpr uint32_t kSwapConsumerRegs = 216;
+static_assert(128 * kSwapProducerRegs + 256 * kSwapConsumerRegs <= 384 * kLaunchRegs, "register split exceeds pool");
+
 template <int STAGES, int NBUF>
 struct alignas(8) SwapState {
   uint64_t full[STAGES];
@@ -219,7 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_wait();
 
   if (warp < 4) {
-    setmaxnreg_dec<kProducerRegs>();
+    setmaxnreg_dec<kSwapProducerRegs>();
     if (warp == 0 && lane == 0) {
       // ------------------------------------------------ TMA producer
       uint32_t it = 0;
@@ -287,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    setmaxnreg_inc<kConsumerRegs>();
+    setmaxnreg_inc<kSwapConsumerRegs>();
     // ------------------------------------------------ promotion + epilogue
     const int ew = threadIdx.x - 128;    // 0..255
     const int ewarp = ew >> 5;           // 0..7
